@@ -1,0 +1,332 @@
+"""LoopVQ oracle: plain fp64 NumPy, CPU only.  TEST INFRASTRUCTURE.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the ``cpu_baseline`` and
+``--impl reference`` legs of ``bench.py`` may import this module.  It shares
+no code with the CUDA library.
+
+Sources (all from the LoopVQ web pages):
+
+* LoopVQ project page (mscheong01.github.io/loopvq), section "Method",
+  figure "Overview of LoopVQ": a code covers G/Tc channels of each of Tc
+  loop steps; one index serves all of them; at inference each loop step reads
+  the shared index through its own slice of the codebook.
+* Same page, "Component 1 -- Loop-axis vector quantization": one index
+  covers channels of several *consecutive* loop steps.
+* Same page, "Serving in SGLang" -- "Write in bf16", "Encode in pages",
+  "Attend from indices": new K/V are written in bf16; the first n_sink and
+  most recent n_recent tokens stay bf16 at every loop step; after every 8
+  generated tokens the oldest recent page is encoded; at loop step t the
+  kernel reads keys/values from the indices through slice B_t and merges with
+  the bf16 attention.
+* Same page, "Results -- Long-context retrieval": n_sink = 64 and
+  n_recent = 256.
+* Same page, "Highlights" and "Efficiency": 0.5 / 0.25 bit per element is
+  32x / 64x compression; bytes read per token and loop step are 8x / 16x
+  fewer than the bf16 keys and values.
+
+Readings taken where the pages are silent (each is stated where it is used):
+one codebook per (Tc-block, KV head, slot); slots are contiguous channel
+groups; a codeword is stored step-major ``[Tc][W]``; Tc-blocks are the
+consecutive steps ``b*Tc .. b*Tc+Tc-1``; plain unweighted L2; ties go to the
+lowest index; the recent window holds ``n_recent + ((ctx - n_sink - n_recent)
+mod page)`` tokens so that the body is whole pages.
+
+Array conventions (all C-order):
+
+* ``X``        keys or values of one layer, ``[T][N][H][D]``
+* ``codebook`` ``[NB][H][J][C][Tc][W]`` with NB = T/Tc, W = G/Tc, J = D/W
+* ``idx``      ``[NB][H][N][J]`` integer codes
+
+Parity: every function here is pinned by ``tests/test_oracle_pins.py``
+(closed forms, hand-worked fixtures under ``tests/golden/``, brute-force and
+library cross-checks, invariants).  No function is "parity unpinned".
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+__all__ = [
+    "geometry",
+    "bits_per_element",
+    "compression_vs_bf16",
+    "bytes_per_token_step",
+    "form_subvectors",
+    "subvector_distances",
+    "encode",
+    "dequantize",
+    "window_split",
+    "attention",
+    "decode_attention",
+    "dense_decode_attention",
+    "reconstruction_mse",
+]
+
+
+# --------------------------------------------------------------------------
+# geometry and accounting
+# --------------------------------------------------------------------------
+
+def geometry(n_loop: int, tc: int, head_dim: int, group_elems: int, n_codes: int = 256) -> dict:
+    """Derived sizes of one loop-axis VQ configuration.
+
+    Project page, "Overview of LoopVQ": a code spans G/Tc channels of each of
+    Tc loop steps.  So W = G/Tc channels per step per code, J = D/W code slots
+    per head, and NB = T/Tc groups of consecutive loop steps.
+    """
+    if tc <= 0 or n_loop % tc:
+        raise ValueError("n_loop must be a multiple of tc")
+    if group_elems % tc:
+        raise ValueError("group_elems must be a multiple of tc")
+    w = group_elems // tc
+    if head_dim % w:
+        raise ValueError("head_dim must be a multiple of group_elems / tc")
+    return {
+        "T": n_loop,
+        "Tc": tc,
+        "NB": n_loop // tc,
+        "G": group_elems,
+        "W": w,
+        "D": head_dim,
+        "J": head_dim // w,
+        "C": n_codes,
+        "bits": bits_per_element(n_codes, group_elems),
+    }
+
+
+def bits_per_element(n_codes: int, group_elems: int) -> float:
+    """An index into n_codes codewords stands for G elements: log2(C)/G bits.
+
+    Project page, "Overview of LoopVQ" (one index serves G elements) and
+    "Highlights" (0.5 and 0.25 bit per element).  Codebooks and the bf16 window
+    are not counted, which is how the pages' 32x / 64x figures come out.
+    """
+    return math.log2(n_codes) / group_elems
+
+
+def compression_vs_bf16(n_codes: int, group_elems: int) -> float:
+    """Ratio of bf16's 16 bits to the quantized bits per element.
+
+    Project page, "Highlights": 32-64x KV cache compression at 0.5 and 0.25 bit.
+    """
+    return 16.0 / bits_per_element(n_codes, group_elems)
+
+
+def bytes_per_token_step(head_dim: int, group_elems: int, tc: int, n_codes: int = 256) -> dict:
+    """Bytes a decode step reads per (token, KV head, loop step).
+
+    bf16 keys and values: 2 tensors x D elements x 2 bytes.  Quantized: one
+    index byte per slot for K and one for V, the index row being read once per
+    loop step (project page, "Serving in SGLang": each loop step reads the
+    shared index row through its own slice).  Project page, "Efficiency":
+    8x fewer bytes at 0.5 bit, 16x at 0.25 bit.
+    """
+    w = group_elems // tc
+    j = head_dim // w
+    index_bytes_per_code = math.ceil(math.log2(n_codes) / 8)
+    bf16 = 2 * head_dim * 2
+    vq = 2 * j * index_bytes_per_code
+    return {"bf16": bf16, "vq": vq, "ratio": bf16 / vq}
+
+
+# --------------------------------------------------------------------------
+# encode
+# --------------------------------------------------------------------------
+
+def form_subvectors(X: np.ndarray, block: int, tc: int, w: int) -> np.ndarray:
+    """Loop-axis sub-vectors of Tc-block ``block``: returns ``[N][H][J][Tc*W]``.
+
+    Project page, "Overview of LoopVQ" and "Component 1": the sub-vector of
+    slot j gathers channels j*W .. j*W+W-1 of each of the Tc consecutive loop
+    steps block*Tc .. block*Tc+Tc-1; element (t, w) sits at position t*W + w.
+    """
+    T, N, H, D = X.shape
+    J = D // w
+    out = np.empty((N, H, J, tc * w), dtype=np.float64)
+    for t in range(tc):
+        step = np.asarray(X[block * tc + t], dtype=np.float64)  # [N][H][D]
+        for j in range(J):
+            out[:, :, j, t * w:(t + 1) * w] = step[:, :, j * w:(j + 1) * w]
+    return out
+
+
+def subvector_distances(x: np.ndarray, codewords: np.ndarray) -> np.ndarray:
+    """Squared L2 distance of every sub-vector to every codeword, by definition.
+
+    ``x`` is ``[n][G]``, ``codewords`` ``[C][G]``; returns ``[n][C]`` with
+    d[i, c] = sum_g (x[i, g] - codewords[c, g])**2, computed from the
+    differences (no ||x||^2 - 2 x.c + ||c||^2 expansion).
+    """
+    x = np.asarray(x, dtype=np.float64)
+    cw = np.asarray(codewords, dtype=np.float64)
+    diff = x[:, None, :] - cw[None, :, :]
+    return np.sum(diff * diff, axis=2)
+
+
+def encode(X: np.ndarray, codebook: np.ndarray, tc: int, chunk: int = 1024):
+    """Brute-force nearest-codeword encoding, ties to the lowest index.
+
+    Project page, "Component 1": each loop-axis sub-vector is replaced by the
+    index of a codeword.  The pages fix no distance; the plain reading is the
+    nearest codeword in unweighted squared L2.  ``np.argmin`` returns the
+    first minimum, i.e. the lowest index on ties.
+
+    Returns ``(idx, d_best, d_second)``, each ``[NB][H][N][J]``; ``d_second``
+    is the second-smallest distance (equal to ``d_best`` on an exact tie) and
+    serves the near-tie tolerance of the parity tests.
+    """
+    T, N, H, D = X.shape
+    NB, H2, J, C, tc2, w = codebook.shape
+    if tc2 != tc or NB * tc != T or H2 != H or J * w != D:
+        raise ValueError("codebook shape does not match X")
+    cb = np.asarray(codebook, dtype=np.float64).reshape(NB, H, J, C, tc * w)
+    idx = np.empty((NB, H, N, J), dtype=np.int64)
+    d_best = np.empty((NB, H, N, J), dtype=np.float64)
+    d_second = np.empty((NB, H, N, J), dtype=np.float64)
+    for b in range(NB):
+        sub = form_subvectors(X, b, tc, w)  # [N][H][J][G]
+        for h in range(H):
+            for j in range(J):
+                for n0 in range(0, N, chunk):
+                    n1 = min(N, n0 + chunk)
+                    d = subvector_distances(sub[n0:n1, h, j], cb[b, h, j])
+                    k = np.argmin(d, axis=1)
+                    idx[b, h, n0:n1, j] = k
+                    d_best[b, h, n0:n1, j] = d[np.arange(n1 - n0), k]
+                    if C > 1:
+                        d_second[b, h, n0:n1, j] = np.partition(d, 1, axis=1)[:, 1]
+                    else:
+                        d_second[b, h, n0:n1, j] = np.inf
+    return idx, d_best, d_second
+
+
+def dequantize(idx: np.ndarray, codebook: np.ndarray, loop_step: int, tc: int) -> np.ndarray:
+    """Reconstruction seen by loop step t: ``[N][H][D]`` in fp64.
+
+    Project page, "Overview of LoopVQ": each loop step reads the shared index
+    through its own slice of the codebook.  Step t belongs to Tc-block
+    b = t // Tc and reads slice t - b*Tc: channel j*W + w of token n is
+    codebook[b][h][j][idx[b][h][n][j]][t - b*Tc][w].
+    """
+    NB, H, J, C, tc2, w = codebook.shape
+    b, tt = divmod(loop_step, tc)
+    N = idx.shape[2]
+    out = np.empty((N, H, J * w), dtype=np.float64)
+    cb = np.asarray(codebook, dtype=np.float64)
+    for h in range(H):
+        for j in range(J):
+            codes = idx[b, h, :, j]
+            if np.any(codes < 0) or np.any(codes >= C):
+                raise ValueError("code out of range")
+            out[:, h, j * w:(j + 1) * w] = cb[b, h, j, codes, tt, :]
+    return out
+
+
+# --------------------------------------------------------------------------
+# decode attention
+# --------------------------------------------------------------------------
+
+def window_split(ctx_len: int, n_sink: int, n_recent: int, page: int):
+    """Split a context of ``ctx_len`` tokens into (sink, body, recent) counts.
+
+    Project page, "Serving in SGLang": the first n_sink and the most recent
+    n_recent tokens stay bf16 at every loop step, and after every 8 generated
+    tokens the oldest recent page is encoded.  Read as: the recent window
+    holds n_recent .. n_recent+page-1 tokens, so the encoded body is whole
+    pages; a context no longer than n_sink + n_recent is all bf16.  The
+    current token is counted in ``ctx_len`` and sits in the recent window.
+    """
+    if ctx_len < 0:
+        raise ValueError("ctx_len must be >= 0")
+    if ctx_len <= n_sink + n_recent:
+        sink = min(ctx_len, n_sink)
+        return sink, 0, ctx_len - sink
+    extra = (ctx_len - n_sink - n_recent) % page if page > 0 else 0
+    recent = n_recent + extra
+    body = ctx_len - n_sink - recent
+    return n_sink, body, recent
+
+
+def attention(q: np.ndarray, K: np.ndarray, V: np.ndarray, scale: float):
+    """Naive softmax attention of one query: returns ``(o, lse)``.
+
+    s_n = scale * q.k_n; o = sum_n exp(s_n - m) v_n / sum_n exp(s_n - m) with
+    m = max_n s_n; lse = m + log(sum_n exp(s_n - m)) (natural log).
+    """
+    q = np.asarray(q, dtype=np.float64)
+    K = np.asarray(K, dtype=np.float64)
+    V = np.asarray(V, dtype=np.float64)
+    if K.shape[0] == 0:
+        return np.zeros(V.shape[1], dtype=np.float64), -np.inf
+    s = scale * (K @ q)
+    m = np.max(s)
+    p = np.exp(s - m)
+    l = np.sum(p)
+    o = (p @ V) / l
+    return o, m + math.log(l)
+
+
+def decode_attention(q, loop_step, tc, idx_k, idx_v, codebook_k, codebook_v,
+                     win_k, win_v, scale):
+    """Decode attention of one request at loop step t over window + body.
+
+    Project page, "Serving in SGLang -- Attend from indices": body keys and
+    values come from the shared indices through slice B_t of the K and V
+    codebooks; the bf16 sink/recent window is used as stored; the two are
+    merged into one softmax.
+
+    q        ``[Hq][D]`` query of loop step t (any float dtype; used in fp64)
+    idx_k/v  ``[NB][H][n_body][J]`` body codes of this request
+    win_k/v  ``[H][n_win][D]`` bf16 window keys/values of loop step t
+    returns  ``(o [Hq][D], lse [Hq])``; query head hq reads KV head
+    hq // (Hq / H).
+    """
+    q = np.asarray(q, dtype=np.float64)
+    Hq, D = q.shape
+    H = codebook_k.shape[1]
+    group = Hq // H
+    Kb = dequantize(idx_k, codebook_k, loop_step, tc)  # [n_body][H][D]
+    Vb = dequantize(idx_v, codebook_v, loop_step, tc)
+    out = np.empty((Hq, D), dtype=np.float64)
+    lse = np.empty(Hq, dtype=np.float64)
+    for hq in range(Hq):
+        h = hq // group
+        K = np.concatenate([np.asarray(win_k[h], dtype=np.float64), Kb[:, h, :]], axis=0)
+        V = np.concatenate([np.asarray(win_v[h], dtype=np.float64), Vb[:, h, :]], axis=0)
+        out[hq], lse[hq] = attention(q[hq], K, V, scale)
+    return out, lse
+
+
+def dense_decode_attention(q, K, V, scale):
+    """Plain decode attention over bf16 keys/values: the dense comparator.
+
+    q ``[Hq][D]``, K/V ``[H][n][D]`` of one loop step; returns (o, lse).
+    """
+    q = np.asarray(q, dtype=np.float64)
+    Hq = q.shape[0]
+    H = K.shape[0]
+    group = Hq // H
+    out = np.empty(q.shape, dtype=np.float64)
+    lse = np.empty(Hq, dtype=np.float64)
+    for hq in range(Hq):
+        out[hq], lse[hq] = attention(q[hq], K[hq // group], V[hq // group], scale)
+    return out, lse
+
+
+def reconstruction_mse(X: np.ndarray, idx: np.ndarray, codebook: np.ndarray, tc: int) -> float:
+    """Mean squared error of the reconstruction over all loop steps and elements.
+
+    Project page, "Method" figure on loop-axis redundancy: at the same bit
+    width, a code spanning four loop steps reconstructs the cache with lower
+    error than a code spanning one step.
+    """
+    T = X.shape[0]
+    acc = 0.0
+    count = 0
+    for t in range(T):
+        Xh = dequantize(idx, codebook, t, tc)
+        diff = np.asarray(X[t], dtype=np.float64) - Xh
+        acc += float(np.sum(diff * diff))
+        count += diff.size
+    return acc / count

@@ -1,0 +1,330 @@
+"""Pins for the CPU oracle: it is checked against things other than itself.
+
+Each test names what fixes the expected value: a figure the LoopVQ pages
+print, a hand-worked fixture (tests/golden/hand_worked.json), a closed form,
+a library routine computing the same definition by another route (SciPy
+cdist, torch scaled_dot_product_attention), or an invariant of softmax
+attention.  Chosen so that a dropped term, a wrong sign or index, or a
+transposed operand anywhere in the oracle fails at least one of them.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+from scipy.spatial.distance import cdist
+from scipy.special import logsumexp
+
+import oracle as O
+from sub_bit_vector_b200 import synth
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _load(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+def _sdpa(q, K, V, scale):
+    """torch's fused attention (math backend, fp64) for one query."""
+    qt = torch.tensor(q, dtype=torch.float64).reshape(1, 1, 1, -1)
+    Kt = torch.tensor(K, dtype=torch.float64).reshape(1, 1, K.shape[0], -1)
+    Vt = torch.tensor(V, dtype=torch.float64).reshape(1, 1, V.shape[0], -1)
+    o = torch.nn.functional.scaled_dot_product_attention(qt, Kt, Vt, scale=scale)
+    return o.reshape(-1).numpy()
+
+
+# ---------------------------------------------------------------- accounting
+
+def test_page_figures_bits_and_bytes():
+    fig = _load("page_figures.json")
+    for row in fig["bits_and_compression"]:
+        assert O.bits_per_element(row["n_codes"], row["group_elems"]) == row["bits"]
+        assert O.compression_vs_bf16(row["n_codes"], row["group_elems"]) == row["compression_vs_bf16"]
+    for row in fig["bytes_per_token_and_loop_step"]:
+        b = O.bytes_per_token_step(row["head_dim"], row["group_elems"], row["tc"])
+        assert b["ratio"] == row["ratio_vs_bf16"]
+    # geometry of the configurations used throughout
+    g = O.geometry(4, 4, 128, 16)
+    assert (g["W"], g["J"], g["NB"], g["bits"]) == (4, 32, 1, 0.5)
+    g = O.geometry(4, 4, 128, 32)
+    assert (g["W"], g["J"], g["NB"], g["bits"]) == (8, 16, 1, 0.25)
+    g = O.geometry(4, 1, 128, 16)
+    assert (g["W"], g["J"], g["NB"]) == (16, 8, 4)
+    with pytest.raises(ValueError):
+        O.geometry(4, 3, 128, 16)
+
+
+# ---------------------------------------------------------- hand-worked case
+
+def test_hand_worked_example():
+    g = _load("hand_worked.json")
+    X = np.array(g["X_T_N_H_D"], dtype=np.float64)
+    cb = np.array(g["codebook_NB_H_J_C_Tc_W"], dtype=np.float64)
+    tc = g["geometry"]["Tc"]
+    idx, d1, d2 = O.encode(X, cb, tc)
+    np.testing.assert_array_equal(idx, np.array(g["idx_NB_H_N_J"]))
+    np.testing.assert_array_equal(d1, np.array(g["d_best_NB_H_N_J"]))
+    np.testing.assert_array_equal(d2, np.array(g["d_second_NB_H_N_J"]))
+    np.testing.assert_array_equal(O.dequantize(idx, cb, 0, tc), np.array(g["dequant_step0_N_H_D"]))
+    np.testing.assert_array_equal(O.dequantize(idx, cb, 1, tc), np.array(g["dequant_step1_N_H_D"]))
+    assert O.reconstruction_mse(X, idx, cb, tc) == g["mse"]
+
+    a = g["attention_step1"]
+    q = np.array([a["q"]])
+    empty = np.zeros((1, 0, 2))
+    o, lse = O.decode_attention(q, 1, tc, idx, idx, cb, cb, empty, empty, a["scale"])
+    np.testing.assert_allclose(o[0], a["o"], rtol=1e-14)
+    assert abs(lse[0] - a["lse"]) < 1e-14
+
+    w = g["attention_step1_with_window"]
+    o, lse = O.decode_attention(q, 1, tc, idx, idx, cb, cb, np.array([w["win_k"]]),
+                                np.array([w["win_v"]]), a["scale"])
+    np.testing.assert_allclose(o[0], w["o"], rtol=1e-14)
+    assert abs(lse[0] - w["lse"]) < 1e-14
+
+
+# -------------------------------------------------------------------- encode
+
+def _subvectors_by_reshape(X, tc, w):
+    """Loop-axis sub-vectors by a second route: reshape D into (J, W) and
+    move the step axis next to W, giving [NB][N][H][J][Tc*W]."""
+    T, N, H, D = X.shape
+    J = D // w
+    Y = X.reshape(T // tc, tc, N, H, J, w)           # [NB][Tc][N][H][J][W]
+    Y = np.moveaxis(Y, 1, 4)                         # [NB][N][H][J][Tc][W]
+    return Y.reshape(T // tc, N, H, J, tc * w)
+
+
+@pytest.mark.parametrize("tc,G", [(4, 16), (4, 32), (1, 16), (2, 8)])
+def test_encode_matches_cdist_argmin(tc, G):
+    rng = np.random.default_rng(11)
+    T, N, H, D, C = 4, 96, 2, 32, 64
+    X = rng.standard_normal((T, N, H, D))
+    w = G // tc
+    cb = rng.standard_normal((T // tc, H, D // w, C, tc, w))
+    idx, d1, d2 = O.encode(X, cb, tc)
+    sub = _subvectors_by_reshape(X, tc, w)
+    for b in range(T // tc):
+        for h in range(H):
+            for j in range(D // w):
+                d = cdist(sub[b, :, h, j], cb[b, h, j].reshape(C, G), "sqeuclidean")
+                np.testing.assert_array_equal(idx[b, h, :, j], np.argmin(d, axis=1))
+                np.testing.assert_allclose(d1[b, h, :, j], d.min(axis=1), rtol=1e-12)
+                np.testing.assert_allclose(d2[b, h, :, j], np.sort(d, axis=1)[:, 1], rtol=1e-12)
+
+
+def test_exact_codeword_returns_its_index_and_roundtrip():
+    rng = np.random.default_rng(5)
+    T, tc, H, D, G, C, N = 4, 4, 2, 16, 16, 32, 40
+    w = G // tc
+    cb = rng.standard_normal((1, H, D // w, C, tc, w))
+    codes = rng.integers(0, C, size=(1, H, N, D // w))
+    X = np.stack([O.dequantize(codes, cb, t, tc) for t in range(T)])   # [T][N][H][D]
+    idx, d1, _ = O.encode(X, cb, tc)
+    np.testing.assert_array_equal(idx, codes)
+    assert np.all(d1 == 0.0)
+    assert O.reconstruction_mse(X, idx, cb, tc) == 0.0
+
+
+def test_duplicate_codewords_give_lowest_index():
+    rng = np.random.default_rng(6)
+    cb = rng.standard_normal((1, 1, 2, 8, 2, 2))
+    cb[0, 0, :, 5] = cb[0, 0, :, 2]      # codeword 5 duplicates 2
+    cb[0, 0, :, 7] = cb[0, 0, :, 2]
+    X = np.zeros((2, 3, 1, 4))
+    for t in range(2):
+        X[t, :, 0, 0:2] = cb[0, 0, 0, 2, t]
+        X[t, :, 0, 2:4] = cb[0, 0, 1, 2, t]
+    idx, d1, d2 = O.encode(X, cb, 2)
+    assert np.all(idx == 2)
+    assert np.all(d1 == 0) and np.all(d2 == 0)
+
+
+def test_tiny_codebook_rows_encode_to_their_own_index():
+    K, _ = synth.tiny_kv(seed=0)
+    tc, G = 4, 16
+    cb = synth.codebook_from_rows(K, tc, G, 256, seed=1)
+    idx, d1, _ = O.encode(K, cb, tc)
+    rng = np.random.Generator(np.random.PCG64(1))
+    rows = rng.permutation(K.shape[1])[:256]       # the draw of slot 0
+    np.testing.assert_array_equal(idx[0, 0, rows, 0], np.arange(256))
+    assert np.all(d1[0, 0, rows, 0] == 0.0)
+
+
+def test_loop_axis_code_beats_single_step_code():
+    """Project page, 'Method', loop-axis redundancy figure: at equal bits a
+    code spanning four loop steps reconstructs with lower error than a code
+    spanning one step.  Directional: the pages print no values."""
+    X = synth.loop_correlated(seed=4, n_loop=4, n_tokens=2048, n_heads=1, head_dim=32,
+                              rho=0.9, bf16=False)
+    mse = {}
+    for tc in (4, 1):
+        cb = synth.codebook_from_rows(X, tc, 16, 256, seed=9)
+        idx, _, _ = O.encode(X, cb, tc)
+        assert O.bits_per_element(256, 16) == 0.5
+        mse[tc] = O.reconstruction_mse(X, idx, cb, tc)
+    assert mse[4] < mse[1]
+
+
+# ----------------------------------------------------------------- attention
+
+def test_window_split_closed_form():
+    assert O.window_split(32768, 64, 256, 8) == (64, 32448, 256)
+    assert O.window_split(32770, 64, 256, 8) == (64, 32448, 258)
+    assert O.window_split(32775, 64, 256, 8) == (64, 32448, 263)
+    assert O.window_split(32776, 64, 256, 8) == (64, 32456, 256)
+    assert O.window_split(320, 64, 256, 8) == (64, 0, 256)
+    assert O.window_split(321, 64, 256, 8) == (64, 0, 257)
+    assert O.window_split(300, 64, 256, 8) == (64, 0, 236)
+    assert O.window_split(50, 64, 256, 8) == (50, 0, 0)
+    assert O.window_split(0, 64, 256, 8) == (0, 0, 0)
+    assert O.window_split(512, 0, 0, 8) == (0, 512, 0)
+    for ctx in range(321, 2000, 37):
+        s, b, r = O.window_split(ctx, 64, 256, 8)
+        assert s + b + r == ctx and b % 8 == 0 and 256 <= r <= 263
+
+
+def test_attention_matches_sdpa_and_logsumexp():
+    rng = np.random.default_rng(2)
+    q = rng.standard_normal(64)
+    K = rng.standard_normal((300, 64))
+    V = rng.standard_normal((300, 64))
+    scale = 1 / 8
+    o, lse = O.attention(q, K, V, scale)
+    np.testing.assert_allclose(o, _sdpa(q, K, V, scale), rtol=1e-12, atol=1e-14)
+    assert abs(lse - logsumexp(scale * K @ q)) < 1e-12
+
+
+def test_all_dense_decode_is_textbook_attention():
+    """Tc = 1, no body (context within the window): plain softmax attention."""
+    rng = np.random.default_rng(3)
+    T, H, D, n = 4, 2, 32, 200
+    Kw = synth.round_bf16(rng.standard_normal((T, H, n, D)))
+    Vw = synth.round_bf16(rng.standard_normal((T, H, n, D)))
+    q = rng.standard_normal((T, H, D))
+    cb = np.zeros((T, H, D // 16, 256, 1, 16))
+    none = np.zeros((T, H, 0, D // 16), dtype=np.int64)
+    for t in range(T):
+        o, _ = O.decode_attention(q[t], t, 1, none, none, cb, cb, Kw[t], Vw[t], D ** -0.5)
+        od, _ = O.dense_decode_attention(q[t], Kw[t], Vw[t], D ** -0.5)
+        for h in range(H):
+            np.testing.assert_allclose(o[h], _sdpa(q[t, h], Kw[t, h], Vw[t, h], D ** -0.5), rtol=1e-12, atol=1e-14)
+            np.testing.assert_allclose(od[h], o[h], rtol=1e-14, atol=1e-15)
+
+
+def test_lossless_vq_equals_dense_attention():
+    """Codebook = every token's own sub-vector, so the body reconstructs
+    exactly and decode attention from codes equals dense attention."""
+    X = synth.loop_correlated(seed=7, n_loop=4, n_tokens=256, n_heads=2, head_dim=32, rho=0.9)
+    V = synth.loop_correlated(seed=8, n_loop=4, n_tokens=256, n_heads=2, head_dim=32, rho=0.9)
+    tc, G = 4, 16
+    cbk = synth.codebook_from_rows(X, tc, G, 256, seed=1)
+    cbv = synth.codebook_from_rows(V, tc, G, 256, seed=2)
+    ik, dk, _ = O.encode(X, cbk, tc)
+    iv, dv, _ = O.encode(V, cbv, tc)
+    assert np.all(dk == 0) and np.all(dv == 0)
+    q = synth.queries(3, 4, 1, 2, 32)[:, 0]
+    # window: the first 16 tokens in bf16, body: the rest from codes
+    for t in range(4):
+        win_k = np.transpose(X[t, :16], (1, 0, 2))
+        win_v = np.transpose(V[t, :16], (1, 0, 2))
+        o, lse = O.decode_attention(q[t], t, tc, ik[:, :, 16:], iv[:, :, 16:], cbk, cbv,
+                                    win_k, win_v, 32 ** -0.5)
+        for h in range(2):
+            ref = _sdpa(q[t, h], X[t, :, h], V[t, :, h], 32 ** -0.5)
+            np.testing.assert_allclose(o[h], ref, rtol=1e-12, atol=1e-13)
+            ref_lse = logsumexp(32 ** -0.5 * X[t, :, h].astype(np.float64) @ q[t, h].astype(np.float64))
+            assert abs(lse[h] - ref_lse) < 1e-11
+
+
+def test_single_token_returns_its_value():
+    rng = np.random.default_rng(4)
+    q = rng.standard_normal((1, 16))
+    k = rng.standard_normal((1, 1, 16))
+    v = rng.standard_normal((1, 1, 16))
+    cb = np.zeros((1, 1, 4, 256, 4, 4))
+    none = np.zeros((1, 1, 0, 4), dtype=np.int64)
+    o, lse = O.decode_attention(q, 0, 4, none, none, cb, cb, k, v, 0.25)
+    np.testing.assert_array_equal(o[0], v[0, 0])
+    assert abs(lse[0] - 0.25 * float(q[0] @ k[0, 0])) < 1e-15
+
+
+def test_shift_of_all_keys_leaves_output_unchanged():
+    """Adding the same vector u to every key (window keys and K codewords)
+    adds scale*q.u to every score, which softmax ignores; lse moves by it."""
+    rng = np.random.default_rng(9)
+    T, tc, H, D, G, C, nb, nw = 4, 4, 1, 16, 16, 16, 50, 10
+    w = G // tc
+    cbk = rng.standard_normal((1, H, D // w, C, tc, w))
+    cbv = rng.standard_normal((1, H, D // w, C, tc, w))
+    ik = rng.integers(0, C, (1, H, nb, D // w))
+    iv = rng.integers(0, C, (1, H, nb, D // w))
+    wk = rng.standard_normal((H, nw, D))
+    wv = rng.standard_normal((H, nw, D))
+    q = rng.standard_normal((H, D))
+    t = 2
+    u = rng.standard_normal(D)
+    cbk2 = cbk.copy()
+    for j in range(D // w):
+        cbk2[0, :, j, :, t, :] += u[j * w:(j + 1) * w]
+    o1, l1 = O.decode_attention(q, t, tc, ik, iv, cbk, cbv, wk, wv, 0.3)
+    o2, l2 = O.decode_attention(q, t, tc, ik, iv, cbk2, cbv, wk + u, wv, 0.3)
+    np.testing.assert_allclose(o1, o2, rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(l2 - l1, 0.3 * q @ u, rtol=1e-11)
+
+
+def test_equal_keys_give_mean_of_values():
+    rng = np.random.default_rng(10)
+    H, D, nb, nw = 2, 8, 30, 5
+    cbk = np.zeros((1, H, 2, 4, 4, 4))
+    cbk[:, :, :, :, :, :] = 0.7                     # all K codewords equal
+    cbv = rng.standard_normal((1, H, 2, 4, 4, 4))
+    ik = rng.integers(0, 4, (1, H, nb, 2))
+    iv = rng.integers(0, 4, (1, H, nb, 2))
+    wk = np.full((H, nw, D), 0.7)
+    wv = rng.standard_normal((H, nw, D))
+    q = rng.standard_normal((H, D))
+    o, lse = O.decode_attention(q, 3, 4, ik, iv, cbk, cbv, wk, wv, 0.5)
+    Vb = O.dequantize(iv, cbv, 3, 4)
+    for h in range(H):
+        mean = np.concatenate([wv[h], Vb[:, h]]).mean(axis=0)
+        np.testing.assert_allclose(o[h], mean, rtol=1e-12, atol=1e-14)
+        assert abs(lse[h] - (0.5 * 0.7 * q[h].sum() + math.log(nb + nw))) < 1e-12
+
+
+def test_gqa_head_mapping():
+    rng = np.random.default_rng(12)
+    H, Hq, D, n = 2, 4, 16, 20
+    K = rng.standard_normal((H, n, D))
+    V = rng.standard_normal((H, n, D))
+    q = rng.standard_normal((Hq, D))
+    o, _ = O.dense_decode_attention(q, K, V, 0.25)
+    for hq in range(Hq):
+        np.testing.assert_allclose(o[hq], _sdpa(q[hq], K[hq // 2], V[hq // 2], 0.25), rtol=1e-12)
+
+
+def test_dequantize_rejects_out_of_range_codes():
+    cb = np.zeros((1, 1, 1, 4, 1, 4))
+    with pytest.raises(ValueError):
+        O.dequantize(np.full((1, 1, 2, 1), 4), cb, 0, 1)
+
+
+# ----------------------------------------------------------------- generator
+
+def test_generator_loop_correlation_and_scale():
+    X = synth.loop_correlated(seed=1, n_loop=4, n_tokens=4096, n_heads=2, head_dim=64,
+                              rho=0.9, bf16=False)
+    a = X[:-1].reshape(3, -1)
+    b = X[1:].reshape(3, -1)
+    for t in range(3):
+        assert abs(np.corrcoef(a[t], b[t])[0, 1] - 0.9) < 0.01
+    assert abs(X.std() - 1.0) < 0.02
+    K = synth.loop_correlated(seed=1, n_loop=4, n_tokens=1024, n_heads=2, head_dim=64,
+                              rho=0.9, n_outlier=4, bf16=True)
+    per_chan = np.abs(K).mean(axis=(0, 1))           # [H][D]
+    assert np.all(np.sort(per_chan, axis=1)[:, -4:].min(axis=1) > 3 * np.median(per_chan))
+    assert np.array_equal(K, synth.round_bf16(K))    # already bf16 values
