@@ -1,0 +1,297 @@
+/*
+ * loopvq.h -- C ABI of libloopvq, the B200 (sm_100a) hot path of LoopVQ:
+ * loop-axis vector-quantized KV-cache encode and decode attention for
+ * looped transformers.
+ *
+ * Method (LoopVQ project page, mscheong01.github.io/loopvq):
+ *   - "Method", figure "Overview of LoopVQ" and "Component 1 -- Loop-axis
+ *     vector quantization": one codebook index covers G/Tc channels of each
+ *     of Tc consecutive loop steps; at inference each loop step reads the
+ *     shared index through its own slice of the codebook.
+ *   - "Serving in SGLang": new keys/values are written in bf16; the first
+ *     n_sink and the most recent n_recent tokens stay bf16 at every loop step
+ *     ("Write in bf16"); after every 8 generated tokens the oldest recent page
+ *     is encoded ("Encode in pages"); at loop step t the attention kernel reads
+ *     keys and values from the indices through slice B_t and merges the result
+ *     with the bf16 attention ("Attend from indices").
+ *   - "Results -- Long-context retrieval": n_sink = 64, n_recent = 256.
+ *
+ * Notation: T loop steps, Tc steps per code, NB = T/Tc code blocks,
+ * H KV heads, Hq query heads (a multiple of H), D head_dim, G elements per
+ * code, W = G/Tc channels per step per code, J = D/W code slots per head,
+ * C <= 256 codewords (one uint8 index).  bits/element = log2(C)/G.
+ *
+ * Conventions for every entry point:
+ *   - The caller owns all memory.  Pointers documented "device" must be
+ *     device (or managed) memory of the current CUDA device; "host" pointers
+ *     are ordinary host memory.  The library allocates nothing and keeps no
+ *     global mutable state; calls on different streams are independent unless
+ *     they share output or workspace buffers.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *     default stream).  Argument errors are detected on the host and returned
+ *     before anything is launched.
+ *   - Faults that only the device can see (a code >= n_codes, a context or
+ *     offset outside the pools) never trap: the kernel sets a bit in the
+ *     workspace's status word, skips the offending work and finishes; read it
+ *     with loopvq_read_device_status().
+ *   - All integer sizes are element counts unless a name ends in _bytes.
+ */
+#ifndef LOOPVQ_H_
+#define LOOPVQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define LOOPVQ_API __attribute__((visibility("default")))
+#else
+#define LOOPVQ_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t, declared without the CUDA headers. */
+typedef struct CUstream_st* loopvq_stream_t;
+
+typedef enum {
+  LOOPVQ_OK = 0,
+  LOOPVQ_ERR_INVALID_ARG = 1,          /* null pointer, bad size, misaligned pointer */
+  LOOPVQ_ERR_UNSUPPORTED = 2,          /* valid geometry that no kernel implements */
+  LOOPVQ_ERR_WORKSPACE_TOO_SMALL = 3,
+  LOOPVQ_ERR_CUDA = 4,                 /* a CUDA runtime call failed (launch, attribute) */
+  LOOPVQ_ERR_DEVICE_FAULT = 5          /* the device status word is non-zero */
+} loopvq_status;
+
+typedef enum { LOOPVQ_F32 = 0, LOOPVQ_BF16 = 1 } loopvq_dtype;
+
+/* Which cache a code stream belongs to; K and V pools use different byte
+ * orders inside a tile (see loopvq_index_pool_bytes). */
+typedef enum { LOOPVQ_KEYS = 0, LOOPVQ_VALUES = 1 } loopvq_kind;
+
+/* Device status word bits (see loopvq_read_device_status). */
+#define LOOPVQ_FAULT_CODE_RANGE   0x1u  /* a K or V code >= n_codes was read */
+#define LOOPVQ_FAULT_CTX_RANGE    0x2u  /* ctx_len > max_ctx_len or < 0 */
+#define LOOPVQ_FAULT_POOL_RANGE   0x4u  /* body/window outside its pool, or misaligned body_off */
+#define LOOPVQ_FAULT_TIMEOUT      0x8u  /* a bounded wait on a copy gave up (never expected) */
+
+/*
+ * One codebook family: K and V of one layer each have their own codebooks of
+ * this shape.  Reading (pages silent): one codebook per (code block b, KV head
+ * h, slot j); slot j covers the contiguous channels j*W .. j*W+W-1.
+ */
+typedef struct {
+  int32_t n_loop;        /* T >= 1 */
+  int32_t tc;            /* Tc >= 1, divides T and G */
+  int32_t n_heads_kv;    /* H >= 1 */
+  int32_t n_heads_q;     /* Hq, a positive multiple of H */
+  int32_t head_dim;      /* D, a multiple of W = G/Tc */
+  int32_t group_elems;   /* G, elements per code */
+  int32_t n_codes;       /* C, 1..256 */
+  loopvq_dtype cb_dtype; /* element type of the codebooks */
+} loopvq_codebook_desc;
+
+/*
+ * Cache layout of one decode batch.  Request r has ctx_len[r] tokens, the
+ * current one included.  They split (project page, "Serving in SGLang") into
+ *   sink   = min(ctx, n_sink) first tokens, bf16;
+ *   body   = whole pages of codes between them;
+ *   recent = n_recent + ((ctx - n_sink - n_recent) mod page) last tokens, bf16;
+ * a context of at most n_sink + n_recent tokens is all bf16 (sink, then recent).
+ * Window pools hold, per request, the sink tokens followed by the recent
+ * tokens (oldest first) at window-pool positions win_off[r] ..; index pools
+ * hold the body at index-pool positions body_off[r] ...
+ */
+typedef struct {
+  int32_t batch;              /* >= 1 */
+  int32_t n_sink;             /* >= 0 (64 on the pages) */
+  int32_t n_recent;           /* >= 0 (256 on the pages) */
+  int32_t page;               /* >= 1 (8 on the pages) */
+  int32_t max_ctx_len;        /* host-side bound on every ctx_len[r]; sizes the launch */
+  int32_t reserved;
+  const int32_t* ctx_len;     /* device [batch] */
+  const int64_t* body_off;    /* device [batch], multiple of 32 */
+  const int64_t* win_off;     /* device [batch] */
+  int64_t body_pool_tokens;   /* capacity of each index pool stream, multiple of 32 */
+  int64_t win_pool_tokens;    /* capacity of each window pool stream */
+} loopvq_cache_layout;
+
+/* ------------------------------------------------------------------ info */
+
+/* Library version string, e.g. "loopvq 0.1.0 sm_100a". */
+LOOPVQ_API const char* loopvq_version(void);
+
+/* Human-readable name of a status code (never NULL). */
+LOOPVQ_API const char* loopvq_status_string(loopvq_status status);
+
+/* Checks a descriptor: LOOPVQ_OK, LOOPVQ_ERR_INVALID_ARG for an inconsistent
+ * one, LOOPVQ_ERR_UNSUPPORTED for a consistent geometry that the decode
+ * kernels do not implement (they need J in {8, 16, 32} and W <= 16). */
+LOOPVQ_API loopvq_status loopvq_validate_desc(const loopvq_codebook_desc* desc);
+
+/* log2(n_codes) / group_elems: bits per quantized element.  Project page,
+ * "Highlights": 0.5 bit (C=256, G=16) and 0.25 bit (C=256, G=32).  Returns a
+ * negative value for an invalid descriptor. */
+LOOPVQ_API float loopvq_bits_per_element(const loopvq_codebook_desc* desc);
+
+/* Host helper: splits a context of ctx_len tokens into (sink, body, recent)
+ * counts by the rule of loopvq_cache_layout, so that callers lay out pools the
+ * way the decode kernel reads them.  Returns LOOPVQ_ERR_INVALID_ARG for
+ * negative sizes, page < 1 or a NULL output. */
+LOOPVQ_API loopvq_status loopvq_ctx_split(int32_t ctx_len, int32_t n_sink, int32_t n_recent, int32_t page,
+                                          int32_t* sink, int32_t* body, int32_t* recent);
+
+/* ------------------------------------------------------------- codebooks */
+
+/*
+ * Size of the packed codebook that the kernels read (0 if desc is invalid).
+ * Packed form, in order: the canonical codebook as given, then per loop step t
+ * the slice B_t re-laid out as [T][H][C][J][W] (code-major), all in cb_dtype.
+ */
+LOOPVQ_API size_t loopvq_codebook_packed_bytes(const loopvq_codebook_desc* desc);
+
+/*
+ * Packs one codebook (K or V of one layer).
+ *   canonical : device, [NB][H][J][C][Tc][W] in cb_dtype; codeword c of
+ *               (b, h, j) holds element (step tt, channel w) at tt*W + w,
+ *               i.e. the loop-axis sub-vector of the project page's
+ *               "Overview of LoopVQ" figure.
+ *   packed    : device, packed_bytes >= loopvq_codebook_packed_bytes(desc),
+ *               16-byte aligned.  Must not overlap canonical.
+ */
+LOOPVQ_API loopvq_status loopvq_codebook_pack(const loopvq_codebook_desc* desc, const void* canonical,
+                                   void* packed, size_t packed_bytes, loopvq_stream_t stream);
+
+/* ------------------------------------------------------------ index pools */
+
+/*
+ * Bytes of one index pool stream of pool_tokens tokens (K or V of one layer):
+ * NB * H * pool_tokens * J, laid out [NB][H][pool_tokens/32][tile], one tile
+ * = 32 tokens x J slots, one uint8 code per (token, slot); the byte order
+ * inside a tile is private to the library and differs between K and V.
+ * pool_tokens must be a positive multiple of 32 (else 0 is returned).
+ */
+LOOPVQ_API size_t loopvq_index_pool_bytes(const loopvq_codebook_desc* desc, int64_t pool_tokens);
+
+/*
+ * Writes plain codes into a pool.  codes: device [NB][H][n_tokens][J] uint8
+ * (token-major, the oracle's order); they go to pool positions
+ * tok_off .. tok_off+n_tokens-1 of every (b, h) stream.  Codes are stored
+ * as given (no range check here; decode checks them).
+ */
+LOOPVQ_API loopvq_status loopvq_index_pool_pack(const loopvq_codebook_desc* desc, loopvq_kind kind,
+                                     const uint8_t* codes, int64_t n_tokens,
+                                     uint8_t* pool, int64_t tok_off, int64_t pool_tokens,
+                                     loopvq_stream_t stream);
+
+/* Inverse of loopvq_index_pool_pack: reads pool positions tok_off .. into
+ * codes [NB][H][n_tokens][J]. */
+LOOPVQ_API loopvq_status loopvq_index_pool_unpack(const loopvq_codebook_desc* desc, loopvq_kind kind,
+                                       const uint8_t* pool, int64_t tok_off, int64_t pool_tokens,
+                                       int64_t n_tokens, uint8_t* codes, loopvq_stream_t stream);
+
+/* ------------------------------------------------------------------ encode */
+
+/*
+ * Loop-axis VQ encode (project page, "Component 1"): for every code block b,
+ * KV head h, slot j and token n, forms the sub-vector
+ *   x[tt*W + w] = X[b*Tc + tt][n][h][j*W + w],  tt < Tc, w < W
+ * and stores argmin_c sum_g (x[g] - codeword_c[g])^2 over c < n_codes, ties
+ * to the lowest c (distances in fp32 from the differences), at pool position
+ * tok_off + n.
+ *   cb_packed : device, from loopvq_codebook_pack (this stream's kind).
+ *   x         : device, element (t, n, h, d) at
+ *               x[t*stride_t + n*stride_n + h*stride_h + d] in x_dtype; d is
+ *               contiguous.  Strides are in elements and must be >= 0.
+ *               E.g. a prefill tensor [T][N][H][D] has strides (N*H*D, H*D, D);
+ *               a window pool [T][H][P][D] has (H*P*D, D, P*D).
+ *   kind      : the stream written (K and V tiles differ in byte order).
+ *   idx_pool  : device, loopvq_index_pool_bytes(desc, pool_tokens) bytes.
+ * n_tokens = 0 is a no-op.  tok_off + n_tokens must not exceed pool_tokens.
+ */
+LOOPVQ_API loopvq_status loopvq_encode(const loopvq_codebook_desc* desc, const void* cb_packed,
+                            loopvq_kind kind, const void* x, loopvq_dtype x_dtype,
+                            int64_t n_tokens, int64_t stride_t, int64_t stride_n,
+                            int64_t stride_h, uint8_t* idx_pool, int64_t tok_off,
+                            int64_t pool_tokens, loopvq_stream_t stream);
+
+/* ---------------------------------------------------------------- decode */
+
+/* Workspace bytes loopvq_decode_attn needs for this layout (0 if invalid). */
+LOOPVQ_API size_t loopvq_decode_workspace_bytes(const loopvq_codebook_desc* desc,
+                                     const loopvq_cache_layout* layout);
+
+/*
+ * Decode attention of loop step `loop_step` for every request and query head
+ * (project page, "Serving in SGLang -- Attend from indices"):
+ *   o = sum_n softmax(softmax_scale * q . k_n) v_n  over the request's tokens,
+ * where window tokens use the bf16 keys/values as stored and body tokens use
+ *   k_n[j*W + w] = B^K_{b,h,j}[idxK[n][j]][t - b*Tc][w],  b = t / Tc
+ * (and v_n likewise from idxV and B^V): the shared index row read through the
+ * step's slice of the codebook.  One softmax covers window and body.
+ *   cbK_packed, cbV_packed : device, packed K and V codebooks.
+ *   idxK_pool, idxV_pool   : device index pools (LOOPVQ_KEYS / LOOPVQ_VALUES
+ *                            byte orders), 16-byte aligned.
+ *   winK, winV             : device bf16 [T][H][win_pool_tokens][D].
+ *   q                      : device [batch][Hq][D] in q_dtype.
+ *   out                    : device [batch][Hq][D] in out_dtype (fp32 keeps
+ *                            the full accuracy; bf16 rounds the result).
+ *   lse_out                : device [batch][Hq] fp32 natural-log
+ *                            log-sum-exp of the scaled scores, or NULL.
+ *   workspace              : device, >= loopvq_decode_workspace_bytes, 256-byte
+ *                            aligned, ZERO-FILLED before its first use; every
+ *                            call leaves it ready for the next one (its split
+ *                            counters return to zero) except the status word,
+ *                            which only loopvq_clear_device_status resets.
+ * Query head hq reads KV head hq / (Hq / H).  A request with ctx_len 0 gets a
+ * zero output and lse -inf.  Calls sharing a workspace must be serialised
+ * (same stream, or ordered by events).
+ */
+LOOPVQ_API loopvq_status loopvq_decode_attn(const loopvq_codebook_desc* desc, const void* cbK_packed,
+                                 const void* cbV_packed, const loopvq_cache_layout* layout,
+                                 const uint8_t* idxK_pool, const uint8_t* idxV_pool,
+                                 const void* winK, const void* winV, const void* q,
+                                 loopvq_dtype q_dtype, int32_t loop_step, float softmax_scale,
+                                 void* out, loopvq_dtype out_dtype, float* lse_out,
+                                 void* workspace, size_t workspace_bytes,
+                                 loopvq_stream_t stream);
+
+/* Waits for `stream`, then reads the workspace status word: LOOPVQ_OK if it
+ * is zero, else LOOPVQ_ERR_DEVICE_FAULT with the LOOPVQ_FAULT_* bits stored
+ * in *bits (if bits is non-NULL). */
+LOOPVQ_API loopvq_status loopvq_read_device_status(const void* workspace, uint32_t* bits,
+                                        loopvq_stream_t stream);
+
+/* Zeroes the status word (asynchronously on stream). */
+LOOPVQ_API loopvq_status loopvq_clear_device_status(void* workspace, loopvq_stream_t stream);
+
+/* -------------------------------------------------- dense bf16 comparator */
+
+/* Workspace bytes of loopvq_dense_decode_attn. */
+LOOPVQ_API size_t loopvq_dense_decode_workspace_bytes(int32_t batch, int32_t n_heads_q, int32_t head_dim,
+                                           int32_t max_ctx_len);
+
+/*
+ * Plain bf16 decode attention with the same split-K structure, used as the
+ * dense comparator (the pages compare against bf16 serving): every token of
+ * request r is read from k/v [H][kv_pool_tokens][D] bf16 (one loop step's
+ * cache) at positions kv_off[r] .. kv_off[r]+ctx_len[r]-1.
+ *   q [batch][Hq][D] in q_dtype, out [batch][Hq][D] fp32, lse_out nullable.
+ *   ctx_len, kv_off : device [batch] (int32, int64).
+ *   workspace: zero-filled before first use, as for loopvq_decode_attn.
+ * D must be 64 or 128.
+ */
+LOOPVQ_API loopvq_status loopvq_dense_decode_attn(int32_t batch, int32_t n_heads_kv, int32_t n_heads_q,
+                                       int32_t head_dim, int32_t max_ctx_len,
+                                       const int32_t* ctx_len, const int64_t* kv_off,
+                                       int64_t kv_pool_tokens, const void* k, const void* v,
+                                       const void* q, loopvq_dtype q_dtype, float softmax_scale,
+                                       float* out, float* lse_out, void* workspace,
+                                       size_t workspace_bytes, loopvq_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LOOPVQ_H_ */

@@ -32,6 +32,10 @@ __all__ = [
     "ragged_context_lengths",
     "queries",
     "uniform_codebook",
+    "key_outlier_channels",
+    "decode_request",
+    "device_codes",
+    "device_normal",
 ]
 
 
@@ -63,7 +67,8 @@ def tiny_kv(seed: int = 0, n_loop: int = 4, n_tokens: int = 512, n_heads: int = 
 
 def loop_correlated(seed: int, n_loop: int, n_tokens: int, n_heads: int, head_dim: int,
                     rho: float = 0.9, n_outlier: int = 0, outlier_scale: float = 8.0,
-                    outlier_dof: float = 4.0, bf16: bool = True) -> np.ndarray:
+                    outlier_dof: float = 4.0, bf16: bool = True,
+                    outlier_channels: np.ndarray | None = None) -> np.ndarray:
     """Ouro-shaped cache tensor ``[T][N][H][D]`` with loop-step correlation rho.
 
     x_0 ~ N(0,1); x_t = rho * x_{t-1} + sqrt(1 - rho^2) * e_t, so every step
@@ -75,8 +80,12 @@ def loop_correlated(seed: int, n_loop: int, n_tokens: int, n_heads: int, head_di
     x = np.empty((n_loop, n_tokens, n_heads, head_dim), dtype=np.float32)
     z0 = rng.standard_normal((n_tokens, n_heads, head_dim)).astype(np.float32)
     chans = None
-    if n_outlier > 0:
+    if outlier_channels is not None:
+        chans = np.asarray(outlier_channels)
+        n_outlier = chans.shape[1]
+    elif n_outlier > 0:
         chans = np.stack([rng.choice(head_dim, size=n_outlier, replace=False) for _ in range(n_heads)])
+    if chans is not None:
         t0 = rng.standard_t(outlier_dof, size=(n_tokens, n_heads, n_outlier)).astype(np.float32)
         for h in range(n_heads):
             z0[:, h, chans[h]] = t0[:, h, :]
@@ -118,14 +127,39 @@ def codebook_from_rows(X: np.ndarray, tc: int, group_elems: int, n_codes: int, s
     return cb
 
 
+def key_outlier_channels(seed: int, n_heads: int, head_dim: int, n_outlier: int = 4) -> np.ndarray:
+    """Seeded choice of ``n_outlier`` heavy-tailed key channels per head: [H][n]."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    return np.stack([rng.choice(head_dim, size=n_outlier, replace=False) for _ in range(n_heads)])
+
+
 def uniform_codebook(seed: int, n_blocks: int, n_heads: int, n_slots: int, n_codes: int,
-                     tc: int, w: int, bf16: bool = True, outlier_scale: float = 1.0) -> np.ndarray:
-    """Random N(0, 1) codebook ``[NB][H][J][C][Tc][W]`` (for large cases that
-    are not encoded from data)."""
+                     tc: int, w: int, bf16: bool = True, outlier_channels: np.ndarray | None = None,
+                     outlier_scale: float = 8.0) -> np.ndarray:
+    """Random N(0, 1) codebook ``[NB][H][J][C][Tc][W]`` for cases whose body
+    codes are drawn directly (too large to encode on the host).  Channels
+    listed in ``outlier_channels`` ([H][n], channel = j*W + w) are scaled by
+    ``outlier_scale``, like the key outlier channels of the cache."""
     rng = np.random.Generator(np.random.PCG64(seed))
     cb = rng.standard_normal((n_blocks, n_heads, n_slots, n_codes, tc, w)).astype(np.float32)
-    cb *= np.float32(outlier_scale)
+    if outlier_channels is not None:
+        for h in range(n_heads):
+            for ch in np.asarray(outlier_channels)[h]:
+                cb[:, h, ch // w, :, :, ch % w] *= np.float32(outlier_scale)
     return round_bf16(cb) if bf16 else cb
+
+
+def decode_request(seed: int, n_loop: int, n_heads: int, head_dim: int, n_slots: int, n_blocks: int,
+                   n_win: int, n_body: int, n_codes: int = 256, rho: float = 0.9,
+                   outlier_channels: np.ndarray | None = None):
+    """One request of a decode batch: bf16 window keys/values
+    ``[T][H][n_win][D]`` (loop-correlated, keys with outlier channels) and
+    body codes ``[NB][H][n_body][J]`` uint8 (uniform)."""
+    wk = loop_correlated(seed, n_loop, n_win, n_heads, head_dim, rho=rho, outlier_channels=outlier_channels)
+    wv = loop_correlated(seed + 7919, n_loop, n_win, n_heads, head_dim, rho=rho)
+    ck = random_codes(seed + 104729, n_blocks, n_heads, n_body, n_slots, n_codes)
+    cv = random_codes(seed + 1299709, n_blocks, n_heads, n_body, n_slots, n_codes)
+    return (np.ascontiguousarray(wk.transpose(0, 2, 1, 3)), np.ascontiguousarray(wv.transpose(0, 2, 1, 3)), ck, cv)
 
 
 def random_codes(seed: int, n_blocks: int, n_heads: int, n_tokens: int, n_slots: int,
@@ -152,3 +186,23 @@ def queries(seed: int, n_loop: int, batch: int, n_heads_q: int, head_dim: int,
     rng = np.random.Generator(np.random.PCG64(seed))
     q = rng.standard_normal((n_loop, batch, n_heads_q, head_dim)).astype(np.float32)
     return round_bf16(q) if bf16 else q
+
+
+# --------------------------------------------------------------------------
+# device-side draws for large benchmark inputs (torch's seeded CUDA RNG);
+# these never feed the oracle
+# --------------------------------------------------------------------------
+
+def device_codes(seed: int, n: int, device="cuda"):
+    """n uniform uint8 codes drawn on the device."""
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    return torch.randint(0, 256, (n,), generator=g, dtype=torch.uint8, device=device)
+
+
+def device_normal(seed: int, shape, dtype=None, device="cuda"):
+    """N(0,1) values drawn on the device, rounded to ``dtype`` (bf16 default)."""
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    x = torch.randn(shape, generator=g, dtype=torch.float32, device=device)
+    return x.to(dtype or torch.bfloat16)

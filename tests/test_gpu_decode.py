@@ -1,0 +1,325 @@
+"""GPU decode attention vs the fp64 oracle, through the C ABI.
+
+Tolerance (the pages fix none; the task's statement is "max relative error
+2e-3 given identical indices"): per (request, query head, loop step) the
+normwise error max_d |o_gpu - o_ref| / max_d |o_ref| <= 2e-3, and the
+natural-log lse within 2e-3.  Both sides consume the same codes, which come
+from the oracle's encoder or the seeded generator, never from the GPU.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from sub_bit_vector_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+TOL = 2e-3
+
+
+def _lib():
+    from sub_bit_vector_b200 import cache, loopvq
+    return cache, loopvq
+
+
+def _err(o, ref):
+    den = np.max(np.abs(ref))
+    return float(np.max(np.abs(o - ref)) / (den if den > 0 else 1.0))
+
+
+class Case:
+    """A decode batch with seeded inputs, held on both sides."""
+
+    def __init__(self, *, seed, ctx_lens, H=16, D=128, G=16, Tc=4, T=4, n_sink=64, n_recent=256, page=8,
+                 Hq=None, n_codes=256, q_dtype=torch.bfloat16, out_dtype=torch.float32,
+                 cb_dtype=torch.bfloat16, max_ctx_len=None, keep=None):
+        cache, L = _lib()
+        self.T, self.Tc, self.H, self.D, self.G = T, Tc, H, D, G
+        self.Hq = Hq or H
+        self.W = G // Tc
+        self.J = D // self.W
+        self.NB = T // Tc
+        self.C = n_codes
+        self.seed = seed
+        self.c = cache.DecodeCache(n_loop=T, tc=Tc, n_heads_kv=H, head_dim=D, group_elems=G, ctx_lens=ctx_lens,
+                                   n_sink=n_sink, n_recent=n_recent, page=page, n_codes=n_codes, n_heads_q=self.Hq,
+                                   cb_dtype=cb_dtype, q_dtype=q_dtype, out_dtype=out_dtype,
+                                   max_ctx_len=max_ctx_len)
+        self.splits = [O.window_split(c, n_sink, n_recent, page) for c in ctx_lens]
+        assert [tuple(s) for s in self.splits] == [tuple(s) for s in self.c.splits]
+        self.outl = synth.key_outlier_channels(seed, H, D)
+        bf = cb_dtype == torch.bfloat16
+        self.cbk = synth.uniform_codebook(seed + 1, self.NB, H, self.J, n_codes, Tc, self.W, bf16=bf,
+                                          outlier_channels=self.outl)
+        self.cbv = synth.uniform_codebook(seed + 2, self.NB, H, self.J, n_codes, Tc, self.W, bf16=bf)
+        self.c.set_codebooks(self.cbk, self.cbv)
+        self.keep = set(range(len(ctx_lens))) if keep is None else set(keep)
+        self.req = {}
+        for r, (s, b, rc) in enumerate(self.splits):
+            data = self.request(r)
+            self.c.set_request_window(r, data[0], data[1])
+            self.c.set_request_codes(r, data[2], data[3])
+            if r in self.keep:
+                self.req[r] = data
+        self.q = synth.queries(seed + 3, T, len(ctx_lens), self.Hq, D, bf16=(q_dtype == torch.bfloat16))
+        torch.cuda.synchronize()
+
+    def request(self, r):
+        s, b, rc = self.splits[r]
+        return synth.decode_request(self.seed * 1000 + r, self.T, self.H, self.D, self.J, self.NB, s + rc, b,
+                                    self.C, outlier_channels=self.outl)
+
+    def run_gpu(self, t):
+        self.c.set_queries(self.q[t])
+        self.c.decode(t)
+        torch.cuda.synchronize()
+        return self.c.out.float().cpu().numpy(), self.c.lse.cpu().numpy()
+
+    def oracle(self, t, r):
+        wk, wv, ck, cv = self.req[r] if r in self.req else self.request(r)
+        return O.decode_attention(self.q[t, r], t, self.Tc, ck, cv, self.cbk, self.cbv, wk[t], wv[t],
+                                  self.D ** -0.5)
+
+    def check(self, t, requests=None, tol=TOL):
+        out, lse = self.run_gpu(t)
+        worst = 0.0
+        for r in (requests if requests is not None else sorted(self.keep)):
+            o_ref, l_ref = self.oracle(t, r)
+            for hq in range(self.Hq):
+                e = _err(out[r, hq], o_ref[hq])
+                worst = max(worst, e)
+                assert e <= tol, f"t={t} r={r} hq={hq} ctx={self.c.ctx_lens[r]} err={e:.3e}"
+                if np.isfinite(l_ref[hq]):
+                    assert abs(lse[r, hq] - l_ref[hq]) <= tol * max(1.0, abs(l_ref[hq])), (t, r, hq)
+                else:
+                    assert lse[r, hq] == -np.inf
+        st, bits = self.c.device_status()
+        assert bits == 0, f"device fault bits {bits:#x}"
+        return worst
+
+
+def test_tiny_decode_from_oracle_codes():
+    """1 layer, 1 head, D=64, 4 loop steps, Tc=4, 512 tokens, fp32, codebook
+    = seeded data rows, codes from the oracle's encoder, no bf16 window."""
+    cache, L = _lib()
+    K, V = synth.tiny_kv(seed=0)
+    cbk = synth.codebook_from_rows(K, 4, 16, 256, seed=1)
+    cbv = synth.codebook_from_rows(V, 4, 16, 256, seed=2)
+    ik, _, _ = O.encode(K, cbk, 4)
+    iv, _, _ = O.encode(V, cbv, 4)
+    c = cache.DecodeCache(n_loop=4, tc=4, n_heads_kv=1, head_dim=64, group_elems=16, ctx_lens=[512], n_sink=0,
+                          n_recent=0, cb_dtype=torch.float32, q_dtype=torch.float32)
+    c.set_codebooks(cbk, cbv)
+    c.set_request_codes(0, ik.astype(np.uint8), iv.astype(np.uint8))
+    q = synth.queries(5, 4, 1, 1, 64, bf16=False)
+    empty = np.zeros((1, 0, 64))
+    for t in range(4):
+        c.set_queries(q[t])
+        c.decode(t)
+        o_ref, l_ref = O.decode_attention(q[t, 0], t, 4, ik, iv, cbk, cbv, empty, empty, 64 ** -0.5)
+        out = c.out.cpu().numpy()[0]
+        assert _err(out[0], o_ref[0]) <= TOL
+        assert abs(c.lse.cpu().numpy()[0, 0] - l_ref[0]) <= TOL
+    assert c.device_status()[1] == 0
+
+
+@pytest.mark.parametrize("t", [0, 1, 2, 3])
+def test_ouro14_32k_half_bit_all_heads(t):
+    """Ouro-1.4B-shaped layer, batch 1, 16 heads x 128, 32768 context, 0.5 bit,
+    bf16 sink 64 + recent 256: every head of every loop step against the oracle."""
+    case = _case_32k()
+    case.check(t)
+
+
+_CACHE = {}
+
+
+def _case_32k():
+    if "32k" not in _CACHE:
+        _CACHE["32k"] = Case(seed=1, ctx_lens=[32768])
+    return _CACHE["32k"]
+
+
+@pytest.mark.parametrize("ctx", [4096, 8192, 16384, 32768, 65536])
+def test_quarter_bit_context_sweep(ctx):
+    """0.25 bit (256 codes over 8 channels x 4 steps), contexts 4K..64K."""
+    case = Case(seed=2, ctx_lens=[ctx], G=32)
+    for t in range(4):
+        case.check(t)
+
+
+def test_batched_ragged_serving_decode_sampled():
+    """Batch 128, Ouro-2.6B-shaped layer (16 x 128, 4 steps, 0.5 bit), context
+    2048 + U{4096..16384} per request: full GPU launch, oracle on a seeded
+    sample of requests (all heads) at every loop step."""
+    ctx = synth.ragged_context_lengths(128)
+    rng = np.random.Generator(np.random.PCG64(77))
+    sample = sorted(set(rng.choice(128, size=6, replace=False).tolist()) | {int(np.argmax(ctx)), int(np.argmin(ctx))})
+    case = Case(seed=3, ctx_lens=ctx.tolist(), keep=sample)
+    for t in range(4):
+        case.check(t, requests=sample)
+
+
+def test_edge_contexts_ragged_gqa():
+    """Empty, single-token, window-only, page-boundary and ragged-tail
+    contexts in one batch, with 2 query heads per KV head."""
+    ctx = [0, 1, 50, 64, 300, 320, 321, 327, 328, 329, 360, 385, 416, 1000, 4421, 9000]
+    case = Case(seed=4, ctx_lens=ctx, H=2, Hq=4)
+    for t in range(4):
+        out, lse = case.run_gpu(t)
+        assert np.all(out[0] == 0) and np.all(lse[0] == -np.inf)
+        case.check(t, requests=[r for r in range(1, len(ctx))])
+
+
+def test_split_boundaries_and_multi_split_merge():
+    """Body lengths around the split length and a context needing the most
+    splits the planner makes for one request."""
+    ctx = [320 + 4064, 320 + 4064 + 8, 320 + 4064 * 2 - 8, 320 + 32, 320 + 24]
+    case = Case(seed=5, ctx_lens=ctx, H=4)
+    for t in (0, 3):
+        case.check(t)
+
+
+@pytest.mark.parametrize("G,D,cbt", [(32, 64, torch.float32), (16, 64, torch.bfloat16), (32, 128, torch.float32),
+                                     (8, 64, torch.float32)])
+def test_other_slot_counts(G, D, cbt):
+    """J = 8, 16 and 32 slot kernels, fp32 and bf16 codebooks, D = 64 / 128."""
+    case = Case(seed=6, ctx_lens=[2000, 777], H=2, D=D, G=G, cb_dtype=cbt)
+    for t in range(4):
+        case.check(t)
+
+
+def test_tc_one_and_two_blocks():
+    """Tc < T: several code blocks, step t reads block t // Tc."""
+    for Tc, G in ((1, 4), (2, 8)):
+        case = Case(seed=7, ctx_lens=[1500], H=2, Tc=Tc, G=G)
+        for t in range(4):
+            case.check(t)
+
+
+def test_bf16_output():
+    case = Case(seed=8, ctx_lens=[3000], H=2, out_dtype=torch.bfloat16)
+    for t in range(2):
+        case.check(t, tol=TOL + 2.0 ** -8)
+
+
+def test_fewer_codes_and_out_of_range_fault():
+    """n_codes < 256 decodes exactly; a code >= n_codes sets the fault bit
+    (the kernel never traps)."""
+    _, L = _lib()
+    case = Case(seed=9, ctx_lens=[1200], H=2, n_codes=100)
+    case.check(0)
+    bad = case.req[0][2].copy()
+    bad[0, 1, 17, 5] = 200
+    case.c.set_request_codes(0, bad, case.req[0][3])
+    case.run_gpu(0)
+    st, bits = case.c.device_status()
+    assert st == L.LOOPVQ_ERR_DEVICE_FAULT and bits & L.LOOPVQ_FAULT_CODE_RANGE
+    case.c.clear_status()
+    assert case.c.device_status()[1] == 0
+    badv = case.req[0][3].copy()
+    badv[0, 0, 3, 2] = 255
+    case.c.set_request_codes(0, case.req[0][2], badv)
+    case.run_gpu(0)
+    assert case.c.device_status()[1] & L.LOOPVQ_FAULT_CODE_RANGE
+
+
+def test_context_beyond_bound_sets_fault():
+    _, L = _lib()
+    case = Case(seed=10, ctx_lens=[900], H=1, max_ctx_len=800)
+    out, lse = case.run_gpu(0)
+    assert case.c.device_status()[1] & L.LOOPVQ_FAULT_CTX_RANGE
+    assert np.all(out == 0)
+
+
+def test_lossless_codes_equal_dense_kernel():
+    """Codebook = every body token's own sub-vector, so the quantized body is
+    exact: LoopVQ decode must equal the dense bf16 kernel on the same cache."""
+    cache, L = _lib()
+    T, Tc, H, D, G, n = 4, 4, 2, 128, 16, 576
+    X = synth.loop_correlated(seed=11, n_loop=T, n_tokens=n, n_heads=H, head_dim=D, n_outlier=4)
+    V = synth.loop_correlated(seed=12, n_loop=T, n_tokens=n, n_heads=H, head_dim=D)
+    s, b, rc = O.window_split(n, 64, 256, 8)
+    assert b == 256
+    cbk = synth.codebook_from_rows(X, Tc, G, 256, seed=13, token_lo=s, token_hi=s + b)
+    cbv = synth.codebook_from_rows(V, Tc, G, 256, seed=14, token_lo=s, token_hi=s + b)
+    ik, dk, _ = O.encode(X[:, s:s + b], cbk, Tc)
+    iv, dv, _ = O.encode(V[:, s:s + b], cbv, Tc)
+    assert np.all(dk == 0) and np.all(dv == 0)
+    c = cache.DecodeCache(n_loop=T, tc=Tc, n_heads_kv=H, head_dim=D, group_elems=G, ctx_lens=[n])
+    c.set_codebooks(cbk, cbv)
+    c.set_request_codes(0, ik.astype(np.uint8), iv.astype(np.uint8))
+    win = np.concatenate([np.arange(s), np.arange(s + b, n)])
+    c.set_request_window(0, X[:, win].transpose(0, 2, 1, 3), V[:, win].transpose(0, 2, 1, 3))
+    kd = torch.from_numpy(X.transpose(0, 2, 1, 3).copy()).cuda().to(torch.bfloat16)   # [T][H][n][D]
+    vd = torch.from_numpy(V.transpose(0, 2, 1, 3).copy()).cuda().to(torch.bfloat16)
+    q = synth.queries(15, T, 1, H, D)
+    ws = torch.zeros(L.loopvq_dense_decode_workspace_bytes(1, H, D, n) + 256, dtype=torch.uint8, device="cuda")
+    ctx = torch.tensor([n], dtype=torch.int32, device="cuda")
+    off = torch.zeros(1, dtype=torch.int64, device="cuda")
+    od = torch.zeros((1, H, D), dtype=torch.float32, device="cuda")
+    ld = torch.zeros((1, H), dtype=torch.float32, device="cuda")
+    for t in range(T):
+        c.set_queries(q[t])
+        c.decode(t)
+        qt = torch.from_numpy(q[t]).cuda().to(torch.bfloat16)
+        L.loopvq_dense_decode_attn(1, H, H, D, n, ctx, off, n, kd[t], vd[t], qt, D ** -0.5, od, ld, ws)
+        torch.cuda.synchronize()
+        ov = c.out.cpu().numpy()[0]
+        odn = od.cpu().numpy()[0]
+        ref, lref = O.dense_decode_attention(q[t, 0], X[t].transpose(1, 0, 2), V[t].transpose(1, 0, 2), D ** -0.5)
+        for h in range(H):
+            assert _err(ov[h], ref[h]) <= TOL
+            assert _err(odn[h], ref[h]) <= TOL
+            assert _err(ov[h], odn[h]) <= 2 * TOL
+
+
+def test_dense_comparator_32k_matches_oracle():
+    """The dense bf16 comparator on the 32K Ouro-1.4B shape."""
+    _, L = _lib()
+    T, H, D, n = 1, 16, 128, 32768
+    K = synth.loop_correlated(seed=21, n_loop=T, n_tokens=n, n_heads=H, head_dim=D, n_outlier=4)[0]
+    V = synth.loop_correlated(seed=22, n_loop=T, n_tokens=n, n_heads=H, head_dim=D)[0]
+    q = synth.queries(23, 1, 1, H, D)[0, 0]
+    kd = torch.from_numpy(K.transpose(1, 0, 2).copy()).cuda().to(torch.bfloat16)
+    vd = torch.from_numpy(V.transpose(1, 0, 2).copy()).cuda().to(torch.bfloat16)
+    ws = torch.zeros(L.loopvq_dense_decode_workspace_bytes(1, H, D, n) + 256, dtype=torch.uint8, device="cuda")
+    od = torch.zeros((1, H, D), dtype=torch.float32, device="cuda")
+    ld = torch.zeros((1, H), dtype=torch.float32, device="cuda")
+    L.loopvq_dense_decode_attn(1, H, H, D, n, torch.tensor([n], dtype=torch.int32, device="cuda"),
+                               torch.zeros(1, dtype=torch.int64, device="cuda"), n, kd, vd,
+                               torch.from_numpy(q[None]).cuda().to(torch.bfloat16), D ** -0.5, od, ld, ws)
+    torch.cuda.synchronize()
+    ref, lref = O.dense_decode_attention(q, K.transpose(1, 0, 2), V.transpose(1, 0, 2), D ** -0.5)
+    o = od.cpu().numpy()[0]
+    for h in range(H):
+        assert _err(o[h], ref[h]) <= TOL
+    np.testing.assert_allclose(ld.cpu().numpy()[0], lref, atol=TOL)
+
+
+def test_repeated_calls_reuse_workspace():
+    """The split counters return to zero: identical results on repeated calls."""
+    case = Case(seed=24, ctx_lens=[5000, 7000], H=2)
+    a, la = case.run_gpu(1)
+    for _ in range(3):
+        b, lb = case.run_gpu(1)
+        np.testing.assert_allclose(a, b, rtol=1e-6, atol=1e-7)
+
+
+def test_host_argument_errors_on_gpu():
+    _, L = _lib()
+    case = Case(seed=25, ctx_lens=[600], H=1)
+    c = case.c
+    with pytest.raises(L.LoopVQError) as e:
+        L.loopvq_decode_attn(c.desc, c.cbK, c.cbV, c.layout, c.idxK, c.idxV, c.winK, c.winV, c.q, 4, 0.1,
+                             c.out, c.lse, c.workspace)
+    assert e.value.status == L.LOOPVQ_ERR_INVALID_ARG
+    with pytest.raises(L.LoopVQError) as e:
+        L.loopvq_decode_attn(c.desc, c.cbK, c.cbV, c.layout, c.idxK, c.idxV, c.winK, c.winV, c.q, 0, 0.1,
+                             c.out, c.lse, c.workspace, workspace_bytes=64)
+    assert e.value.status == L.LOOPVQ_ERR_WORKSPACE_TOO_SMALL
+    with pytest.raises(L.LoopVQError) as e:
+        L.loopvq_decode_attn(c.desc, c.cbK, c.cbV, c.layout, c.idxK[1:], c.idxV, c.winK, c.winV, c.q, 0, 0.1,
+                             c.out, c.lse, c.workspace)
+    assert e.value.status == L.LOOPVQ_ERR_INVALID_ARG
