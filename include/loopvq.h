@@ -257,6 +257,37 @@ LOOPVQ_API loopvq_status loopvq_decode_attn(const loopvq_codebook_desc* desc, co
                                  void* workspace, size_t workspace_bytes,
                                  loopvq_stream_t stream);
 
+/*
+ * Allocation-free variant of loopvq_decode_attn (the LoopVQ pages have no
+ * counterpart; this is a packaging choice of the library).
+ *
+ * For callers that cannot allocate device memory: a plugin running inside a
+ * host process whose allocator owns the GPU's memory, or a latency-critical
+ * path that must not call cudaMalloc (it synchronizes the device).  Arguments
+ * and results are those of loopvq_decode_attn, except that there is no
+ * workspace: the split partials and counters live in a fixed 8 MiB array
+ * inside the library's device image, present on every GPU that loads the
+ * library until the process exits.  Nothing is allocated or freed here.
+ *   fault_bits : device uint32 that receives the LOOPVQ_FAULT_* bits of this
+ *                call (OR-ed in; the caller zeroes it), or NULL to drop them.
+ * Returns LOOPVQ_ERR_WORKSPACE_TOO_SMALL when the layout would need more than
+ * the 8 MiB array (loopvq_decode_workspace_bytes tells how much it needs).
+ * The first call on a device looks up the array's device address (a
+ * cudaGetSymbolAddress with that device current); make that first call
+ * before any stream capture.  Every call shares the one array per device:
+ * each call zeroes its counters on `stream` before the kernel runs, and two
+ * calls whose kernels overlap on the GPU (different streams, no ordering)
+ * race on it and give wrong results.
+ */
+LOOPVQ_API loopvq_status loopvq_decode_attn_noalloc(const loopvq_codebook_desc* desc, const void* cbK_packed,
+                                                    const void* cbV_packed, const loopvq_cache_layout* layout,
+                                                    const uint8_t* idxK_pool, const uint8_t* idxV_pool,
+                                                    const void* winK, const void* winV, const void* q,
+                                                    loopvq_dtype q_dtype, int32_t loop_step,
+                                                    float softmax_scale, void* out, loopvq_dtype out_dtype,
+                                                    float* lse_out, uint32_t* fault_bits,
+                                                    loopvq_stream_t stream);
+
 /* Waits for `stream`, then reads the workspace status word: LOOPVQ_OK if it
  * is zero, else LOOPVQ_ERR_DEVICE_FAULT with the LOOPVQ_FAULT_* bits stored
  * in *bits (if bits is non-NULL). */

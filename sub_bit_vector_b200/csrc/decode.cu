@@ -678,3 +678,136 @@ extern "C" loopvq_status loopvq_decode_attn(const loopvq_codebook_desc* desc, co
 #undef LOOPVQ_LAUNCH
   return cudaGetLastError() == cudaSuccess ? LOOPVQ_OK : LOOPVQ_ERR_CUDA;
 }
+
+// ---------------------------------------------------------------------------
+// Allocation-free variant of loopvq_decode_attn.
+//
+// Some callers cannot hand the library a workspace: a plugin loaded into a
+// host process whose allocator owns all device memory, or a latency-critical
+// path where cudaMalloc (which synchronizes the device) is not allowed.  This
+// variant keeps the split partials and counters in a fixed array that lives
+// in the library's own device image, so the caller supplies only inputs and
+// outputs.  The array is kLoopvqStaticScratchBytes per device and stays
+// resident on every GPU that loads the library until the process exits.
+// ---------------------------------------------------------------------------
+
+#include <mutex>
+
+namespace loopvq {
+
+constexpr size_t kLoopvqStaticScratchBytes = 8u << 20;  // 8 MiB
+static __device__ __align__(256) unsigned char g_decode_scratch[kLoopvqStaticScratchBytes];
+
+constexpr int kMaxDevices = 64;
+static std::mutex g_scratch_mutex;
+static void* g_scratch_addr[kMaxDevices];
+
+// Device address of g_decode_scratch on the current device.  In host code the
+// symbol is only a host-side stand-in, so the real address is looked up once
+// per device (with that device current) and cached.
+static loopvq_status static_scratch(void** addr) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return LOOPVQ_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return LOOPVQ_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_scratch_mutex);
+  if (!g_scratch_addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_decode_scratch) != cudaSuccess || p == nullptr) {
+      cudaGetLastError();
+      return LOOPVQ_ERR_CUDA;
+    }
+    g_scratch_addr[dev] = p;
+  }
+  *addr = g_scratch_addr[dev];
+  return LOOPVQ_OK;
+}
+
+}  // namespace loopvq
+
+extern "C" loopvq_status loopvq_decode_attn_noalloc(const loopvq_codebook_desc* desc, const void* cbK_packed,
+                                                    const void* cbV_packed, const loopvq_cache_layout* layout,
+                                                    const uint8_t* idxK_pool, const uint8_t* idxV_pool,
+                                                    const void* winK, const void* winV, const void* q,
+                                                    loopvq_dtype q_dtype, int32_t loop_step, float softmax_scale,
+                                                    void* out, loopvq_dtype out_dtype, float* lse_out,
+                                                    uint32_t* fault_bits, loopvq_stream_t stream) {
+  Geo g;
+  loopvq_status st = make_geo(desc, &g);
+  if (st != LOOPVQ_OK) return st;
+  if ((st = check_layout(layout)) != LOOPVQ_OK) return st;
+  if (g.J != 8 && g.J != 16 && g.J != 32) return LOOPVQ_ERR_UNSUPPORTED;
+  if (g.D != 64 && g.D != 128) return LOOPVQ_ERR_UNSUPPORTED;
+  if (loop_step < 0 || loop_step >= g.T) return LOOPVQ_ERR_INVALID_ARG;
+  if (q_dtype != LOOPVQ_F32 && q_dtype != LOOPVQ_BF16) return LOOPVQ_ERR_INVALID_ARG;
+  if (out_dtype != LOOPVQ_F32 && out_dtype != LOOPVQ_BF16) return LOOPVQ_ERR_INVALID_ARG;
+  if (!(softmax_scale == softmax_scale)) return LOOPVQ_ERR_INVALID_ARG;
+  if (!cbK_packed || !cbV_packed || !idxK_pool || !idxV_pool || !winK || !winV || !q || !out)
+    return LOOPVQ_ERR_INVALID_ARG;
+  if (((uintptr_t)idxK_pool & 15) || ((uintptr_t)idxV_pool & 15) || ((uintptr_t)winK & 15) ||
+      ((uintptr_t)winV & 15) || ((uintptr_t)cbK_packed & 15) || ((uintptr_t)cbV_packed & 15) ||
+      ((uintptr_t)fault_bits & 3))
+    return LOOPVQ_ERR_INVALID_ARG;
+  const WsLayout ws = decode_ws(g, layout);
+  if (ws.total > kLoopvqStaticScratchBytes) return LOOPVQ_ERR_WORKSPACE_TOO_SMALL;
+  const int64_t units = (int64_t)layout->batch * g.Hq;
+  const DecodePlan pl = decode_plan(units, max_body_tokens(layout), device_sm_count());
+  if (units > 65535LL * 65535LL || pl.max_splits > 1 << 20 || layout->batch > 65535 || g.Hq > 65535)
+    return LOOPVQ_ERR_UNSUPPORTED;
+
+  void* scratch = nullptr;
+  if ((st = static_scratch(&scratch)) != LOOPVQ_OK) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  // the status word and the split counters must start at zero
+  if (cudaMemsetAsync(scratch, 0, ws.partials_off, s) != cudaSuccess) return LOOPVQ_ERR_CUDA;
+
+  DecodeParams p;
+  p.T = g.T; p.Tc = g.Tc; p.H = g.H; p.Hq = g.Hq; p.D = g.D; p.J = g.J; p.W = g.W; p.C = g.C;
+  p.loop_step = loop_step;
+  p.scale_log2 = softmax_scale * 1.4426950408889634f;
+  p.batch = layout->batch; p.n_sink = layout->n_sink; p.n_recent = layout->n_recent;
+  p.page = layout->page; p.max_ctx = layout->max_ctx_len;
+  p.ctx_len = layout->ctx_len; p.body_off = layout->body_off; p.win_off = layout->win_off;
+  p.body_pool_tokens = layout->body_pool_tokens; p.win_pool_tokens = layout->win_pool_tokens;
+  const size_t eb = cb_elem_bytes(g);
+  const size_t step_off = packed_slices_offset_bytes(g) + (size_t)loop_step * slice_elems_per_step(g) * eb;
+  p.cbK_slice = (const uint8_t*)cbK_packed + step_off;
+  p.cbV_slice = (const uint8_t*)cbV_packed + step_off;
+  const size_t blk_bytes = (size_t)g.H * layout->body_pool_tokens * g.J;
+  p.idxK = idxK_pool + (loop_step / g.Tc) * blk_bytes;
+  p.idxV = idxV_pool + (loop_step / g.Tc) * blk_bytes;
+  const size_t win_step = (size_t)g.H * layout->win_pool_tokens * g.D;
+  p.winK = (const __nv_bfloat16*)winK + loop_step * win_step;
+  p.winV = (const __nv_bfloat16*)winV + loop_step * win_step;
+  p.q = q; p.q_bf16 = q_dtype == LOOPVQ_BF16;
+  p.out = out; p.out_bf16 = out_dtype == LOOPVQ_BF16; p.lse = lse_out;
+  p.status = fault_bits ? fault_bits : (uint32_t*)scratch;
+  p.tickets = (uint32_t*)((uint8_t*)scratch + ws.tickets_off);
+  p.partials = (float*)((uint8_t*)scratch + ws.partials_off);
+  p.split_len = pl.split_len;
+  p.max_splits = pl.max_splits;
+
+  dim3 grid(pl.max_splits, g.Hq, layout->batch);
+#define LOOPVQ_LAUNCH(JJ, DD, CBT)                                                                    \
+  do {                                                                                               \
+    auto kfn = decode_kernel<JJ, DD, CBT>;                                                           \
+    if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, kDynSmem) != cudaSuccess) \
+      return LOOPVQ_ERR_CUDA;                                                                        \
+    kfn<<<grid, kThreads, kDynSmem, s>>>(p);                                                         \
+  } while (0)
+#define LOOPVQ_LAUNCH_J(DD, CBT)                      \
+  do {                                                \
+    if (g.J == 32) LOOPVQ_LAUNCH(32, DD, CBT);        \
+    else if (g.J == 16) LOOPVQ_LAUNCH(16, DD, CBT);   \
+    else LOOPVQ_LAUNCH(8, DD, CBT);                   \
+  } while (0)
+  if (g.D == 128) {
+    if (g.cb_bf16) LOOPVQ_LAUNCH_J(128, __nv_bfloat16);
+    else LOOPVQ_LAUNCH_J(128, float);
+  } else {
+    if (g.cb_bf16) LOOPVQ_LAUNCH_J(64, __nv_bfloat16);
+    else LOOPVQ_LAUNCH_J(64, float);
+  }
+#undef LOOPVQ_LAUNCH_J
+#undef LOOPVQ_LAUNCH
+  return cudaGetLastError() == cudaSuccess ? LOOPVQ_OK : LOOPVQ_ERR_CUDA;
+}

@@ -37,7 +37,8 @@ EXPORTED = [
     "loopvq_bits_per_element",
     "loopvq_codebook_packed_bytes", "loopvq_codebook_pack", "loopvq_index_pool_bytes",
     "loopvq_index_pool_pack", "loopvq_index_pool_unpack", "loopvq_encode",
-    "loopvq_decode_workspace_bytes", "loopvq_decode_attn", "loopvq_read_device_status",
+    "loopvq_decode_workspace_bytes", "loopvq_decode_attn", "loopvq_decode_attn_noalloc",
+    "loopvq_read_device_status",
     "loopvq_clear_device_status", "loopvq_dense_decode_workspace_bytes", "loopvq_dense_decode_attn",
 ]
 
@@ -85,6 +86,8 @@ def _load() -> ctypes.CDLL:
         "loopvq_decode_workspace_bytes": (SZ, [D, L]),
         "loopvq_decode_attn": (ctypes.c_int, [D, P, P, L, U8P, U8P, P, P, P, ctypes.c_int, I32, F, P,
                                               ctypes.c_int, P, P, SZ, P]),
+        "loopvq_decode_attn_noalloc": (ctypes.c_int, [D, P, P, L, U8P, U8P, P, P, P, ctypes.c_int, I32, F, P,
+                                                      ctypes.c_int, P, P, P]),
         "loopvq_read_device_status": (ctypes.c_int, [P, ctypes.POINTER(ctypes.c_uint32), P]),
         "loopvq_clear_device_status": (ctypes.c_int, [P, P]),
         "loopvq_dense_decode_workspace_bytes": (SZ, [I32, I32, I32, I32]),
@@ -220,6 +223,18 @@ def loopvq_decode_attn(desc, cbK_packed, cbV_packed, layout, idxK_pool, idxV_poo
         ctypes.byref(desc), _ptr(cbK_packed), _ptr(cbV_packed), ctypes.byref(layout), _ptr(idxK_pool),
         _ptr(idxV_pool), _ptr(winK), _ptr(winV), _ptr(q), _dtype_code(q), loop_step, softmax_scale,
         _ptr(out), _dtype_code(out), _ptr(lse_out), _ptr(workspace), wb, _stream(stream)))
+
+
+def loopvq_decode_attn_noalloc(desc, cbK_packed, cbV_packed, layout, idxK_pool, idxV_pool, winK, winV, q,
+                               loop_step, softmax_scale, out, lse_out, fault_bits=None, stream=None) -> None:
+    """Same as loopvq_decode_attn but with no workspace: for callers that
+    cannot allocate device memory (the library's fixed per-device scratch is
+    used; calls must not overlap on the GPU).  ``fault_bits`` is an optional
+    one-element uint32/int32 device tensor that receives the fault bits."""
+    _check("loopvq_decode_attn_noalloc", _lib.loopvq_decode_attn_noalloc(
+        ctypes.byref(desc), _ptr(cbK_packed), _ptr(cbV_packed), ctypes.byref(layout), _ptr(idxK_pool),
+        _ptr(idxV_pool), _ptr(winK), _ptr(winV), _ptr(q), _dtype_code(q), loop_step, softmax_scale,
+        _ptr(out), _dtype_code(out), _ptr(lse_out), _ptr(fault_bits), _stream(stream)))
 
 
 def loopvq_read_device_status(workspace, stream=None):
