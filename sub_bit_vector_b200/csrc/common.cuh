@@ -31,16 +31,19 @@ inline size_t packed_slices_offset_bytes(const Geo& g) {
 
 // ------------------------------------------------------------ pool layout
 // A pool stream is [NB][H][pool_tokens/32][tile]; a tile holds 32 tokens x J
-// slots.  Inside a tile lane l = g*J + j (g = token / J, j = slot) owns J
-// consecutive bytes; for V byte i of the lane is token g*J + i, for K it is
-// token g*J + (i ^ j).  The K order lets the decode kernel sum the per-slot
-// partial scores with a select-free butterfly (each lane holds token i^j in
-// register i, so every exchange sends the upper half of its registers).
+// slots, one uint8 code each.  Token n of a tile is read by lane n of a warp
+// in 16-byte pieces (one piece for J <= 16, two for J = 32): piece p of token
+// n sits at p*512 + n*min(J,16), so each warp-wide piece load is one
+// contiguous 512-byte (or 256-byte) run.  Inside a token's J bytes the codes
+// are rotated: byte s holds slot (s + n) mod J.  At step s of the decode loops
+// the 32 lanes therefore touch 32 different slots, i.e. 32 different shared
+// memory banks of the per-slot lookup tables and histograms.  K and V tiles
+// use the same order.
 __host__ __device__ inline int64_t tile_byte(int J, int kind, int n_in_tile, int j) {
-  int g = n_in_tile / J, i = n_in_tile % J;
-  int lane = g * J + j;
-  int pos = (kind == LOOPVQ_KEYS) ? (i ^ j) : i;
-  return (int64_t)lane * J + pos;
+  (void)kind;
+  const int s = ((j - n_in_tile) % J + J) % J;
+  const int piece = J < 16 ? J : 16;
+  return (int64_t)(s / piece) * (32 * piece) + (int64_t)n_in_tile * piece + (s % piece);
 }
 __host__ __device__ inline int64_t pool_byte(int J, int kind, int64_t pool_tokens, int b, int H, int h,
                                              int64_t n, int j) {
@@ -148,33 +151,64 @@ __device__ __forceinline__ void set_fault(uint32_t* status, uint32_t bits) {
 
 // Combine of split partials for one (request, query head): the last split to
 // finish merges every split's (o[D], m, l) by log-sum-exp; m is in log2 units
-// and o is unnormalised (sum of weights 2^(s - m) times values).  Called by
-// every thread of the CTA; threads d < D each produce one output channel.
-__device__ __forceinline__ void combine_splits(const float* part, int n_splits, int D, void* out,
-                                               int out_bf16, float* lse) {
+// and o is unnormalised (sum of weights 2^(s - m) times values).  All loads of
+// a phase are independent so they are in flight together: phase 1 stages
+// every split's (m, l) in shared memory, phase 2 has nthr/D threads per
+// output channel each summing a stride of the splits, phase 3 adds those up.
+// `sm` holds 2*kMaxCombineSplits + nthr floats; `sync` is the CTA barrier of
+// the nthr participating threads (tid in [0, nthr)).
+constexpr int kMaxCombineSplits = 1024;
+struct BlockSync {
+  __device__ __forceinline__ void operator()() const { __syncthreads(); }
+};
+template <typename Sync>
+__device__ __forceinline__ void combine_splits(const float* part, int n_splits, int D, void* out, int out_bf16,
+                                               float* lse, float* sm, int tid, int nthr, Sync sync) {
+  float* sm_m = sm;
+  float* sm_l = sm + kMaxCombineSplits;
+  float* sm_acc = sm + 2 * kMaxCombineSplits;
+  const size_t stride = (size_t)(D + 4);
+  for (int s = tid; s < n_splits; s += nthr) {
+    sm_m[s] = __ldcg(part + s * stride + D);
+    sm_l[s] = __ldcg(part + s * stride + D + 1);
+  }
+  sync();
   float M = -INFINITY;
-  for (int s = 0; s < n_splits; ++s) M = fmaxf(M, __ldcg(part + (size_t)s * (D + 4) + D));
+  for (int s = 0; s < n_splits; ++s) M = fmaxf(M, sm_m[s]);
   float L = 0.f;
-  for (int s = 0; s < n_splits; ++s) {
-    float ms = __ldcg(part + (size_t)s * (D + 4) + D);
-    if (ms != -INFINITY) L += __ldcg(part + (size_t)s * (D + 4) + D + 1) * exp2f(ms - M);
-  }
-  for (int d = threadIdx.x; d < D; d += blockDim.x) {
-    float acc = 0.f;
-    if (M != -INFINITY) {
-      for (int s = 0; s < n_splits; ++s) {
-        float ms = __ldcg(part + (size_t)s * (D + 4) + D);
-        if (ms != -INFINITY) acc += __ldcg(part + (size_t)s * (D + 4) + d) * exp2f(ms - M);
-      }
-      acc = L > 0.f ? acc / L : 0.f;
+  for (int s = 0; s < n_splits; ++s)
+    if (sm_m[s] != -INFINITY) L += sm_l[s] * exp2f(sm_m[s] - M);
+  const int P = nthr / D;
+  const int d = tid % D, pi = tid / D;
+  float acc = 0.f;
+  if (pi < P && M != -INFINITY) {
+    int s = pi;
+    for (; s + 3 * P < n_splits; s += 4 * P) {
+      const float a0 = __ldcg(part + s * stride + d);
+      const float a1 = __ldcg(part + (s + P) * stride + d);
+      const float a2 = __ldcg(part + (s + 2 * P) * stride + d);
+      const float a3 = __ldcg(part + (s + 3 * P) * stride + d);
+      const float w0 = sm_m[s] != -INFINITY ? exp2f(sm_m[s] - M) : 0.f;
+      const float w1 = sm_m[s + P] != -INFINITY ? exp2f(sm_m[s + P] - M) : 0.f;
+      const float w2 = sm_m[s + 2 * P] != -INFINITY ? exp2f(sm_m[s + 2 * P] - M) : 0.f;
+      const float w3 = sm_m[s + 3 * P] != -INFINITY ? exp2f(sm_m[s + 3 * P] - M) : 0.f;
+      acc = fmaf(a0, w0, fmaf(a1, w1, fmaf(a2, w2, fmaf(a3, w3, acc))));
     }
-    if (out_bf16)
-      ((__nv_bfloat16*)out)[d] = __float2bfloat16_rn(acc);
-    else
-      ((float*)out)[d] = acc;
+    for (; s < n_splits; s += P)
+      if (sm_m[s] != -INFINITY) acc = fmaf(__ldcg(part + s * stride + d), exp2f(sm_m[s] - M), acc);
   }
-  if (lse && threadIdx.x == 0)
-    *lse = (M == -INFINITY || !(L > 0.f)) ? -INFINITY : (M + log2f(L)) * 0.6931471805599453f;
+  if (pi < P) sm_acc[pi * D + d] = acc;
+  sync();
+  if (tid < D) {
+    float o = 0.f;
+    for (int i = 0; i < P; ++i) o += sm_acc[i * D + tid];
+    o = (M != -INFINITY && L > 0.f) ? o / L : 0.f;
+    if (out_bf16)
+      ((__nv_bfloat16*)out)[tid] = __float2bfloat16_rn(o);
+    else
+      ((float*)out)[tid] = o;
+  }
+  if (lse && tid == 0) *lse = (M == -INFINITY || !(L > 0.f)) ? -INFINITY : (M + log2f(L)) * 0.6931471805599453f;
 }
 
 }  // namespace loopvq

@@ -7,19 +7,19 @@
 //
 //   window split : the bf16 sink + recent tokens, online softmax in fp32.
 //   body split   : up to kSplitCap tokens of codes, in two passes over a
-//                  TMA-fed shared-memory ring:
+//                  TMA-fed shared-memory ring (4 x 32 KB in flight):
 //     pass K  -- score s_n = sum_j LUT[j][idxK[n][j]] with the per-step
-//                lookup table LUT[j][c] = scale*log2(e) * q_j . B^K_t[c][j];
-//                lane l owns slot l%J, so a warp-wide gather touches 32
-//                distinct banks; the J partial sums of a token are added by
-//                a select-free butterfly (the K tile byte order puts token
-//                i^j in register i of lane j).
+//                lookup table LUT[j][c] = scale*log2(e) * q_j . B^K_t[c][j].
+//                Lane l of a warp owns token l of a 32-token tile and walks
+//                its slots in the tile's rotated order (slot (s+l) mod J at
+//                step s), so every warp-wide gather hits 32 distinct banks
+//                and no cross-lane reduction is needed.
 //     pass V  -- with the split maximum m known, token weight
 //                p_n = 2^(s_n - m) in (0, 1] becomes a u32 fixed-point
 //                q_n = floor(p_n 2^S + u_n) (u_n a Weyl dither, so the
 //                rounding is unbiased) and is added into a per-slot 256-bin
 //                histogram hist[j][idxV[n][j]] with shared-memory integer
-//                atomics (one bank per lane, conflict free);
+//                atomics (same rotation: conflict free).
 //     epilogue   -- o[jW+w] = 2^-S sum_c hist[j][c] B^V_t[c][j][w].
 //   The last CTA of a (request, head) merges the splits' (m, l, o) by
 //   log-sum-exp (atomic ticket, no waiting).
@@ -37,13 +37,21 @@ namespace loopvq {
 constexpr int kNW = 16;                      // consumer warps
 constexpr int kThreads = (kNW + 1) * 32;     // + one producer warp
 constexpr int kStages = 4;
-constexpr int kStageBytes = 16384;
+constexpr int kStageBytes = 32768;
 constexpr int kSplitCap = 4064;              // max body tokens per split, multiple of 32
-constexpr int kRegionAlign = 32768;          // LUT / histogram base alignment
-// dynamic smem: alignment pad + LUT (32 KB) + histogram (32 KB) + ring + scores + misc
+// The lookup table and the histogram share one 64 KB region of 256 rows (one
+// per code) of 256 bytes: 32 fp32 table columns, then 32 u32 histogram
+// columns.  The region is 64 KB aligned in the shared window, so the shared
+// address of (code, column) is a single byte permute: code in byte 1, the
+// column offset in byte 0, the region base in bytes 2-3.
+constexpr int kRegionBytes = 65536;
+constexpr int kHistColOff = 128;             // histogram column offset in a row
 constexpr int kScoresBytes = kSplitCap * 4;
 constexpr int kMiscBytes = 4096;
-constexpr int kDynSmem = kRegionAlign + 32768 + 32768 + kStages * kStageBytes + kScoresBytes + kMiscBytes;
+// allocation: the region, the ring, scores and misc, plus room to align the
+// region to 64 KB (the part below the region holds misc, scores and ring
+// stages that fit there)
+constexpr int kDynSmem = 228352;
 
 struct DecodeParams {
   int T, Tc, H, Hq, D, J, W, C;
@@ -75,74 +83,105 @@ struct DecodeParams {
 __device__ __forceinline__ void consumer_sync() {
   asm volatile("bar.sync 1, %0;" ::"n"(kNW * 32) : "memory");
 }
+struct ConsumerSync {
+  __device__ __forceinline__ void operator()() const { consumer_sync(); }
+};
 
-// Shared address of the LUT / histogram entry of `code` (byte K of w) for
-// this lane: rows of 32 words, column = lane.  base is 32 KB aligned, so the
-// row offset can be OR-ed in.
-template <int K>
-__device__ __forceinline__ uint32_t code_addr(uint32_t w, uint32_t base) {
-  uint32_t x = (K == 0) ? (w << 7) : (w >> (8 * K - 7));
-  return (x & 0x7F80u) | base;
-}
 __device__ __forceinline__ float lds_f32(uint32_t a) {
   float v;
   asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(a));
   return v;
 }
-__device__ __forceinline__ void red_add_u32(uint32_t a, uint32_t v) {
-  asm volatile("red.shared.add.u32 [%0], %1;" ::"r"(a), "r"(v) : "memory");
+// the histogram bin sits kHistColOff bytes after the table entry of the same
+// code and column
+__device__ __forceinline__ void red_hist_u32(uint32_t lut_addr, uint32_t v) {
+  asm volatile("red.shared.add.u32 [%0+128], %1;" ::"r"(lut_addr), "r"(v) : "memory");
+}
+// acc (two packed fp32) += (x, y)
+__device__ __forceinline__ uint64_t add_f32x2(uint64_t acc, float x, float y) {
+  uint64_t r;
+  asm("{\n .reg .b64 t;\n mov.b64 t, {%2, %3};\n add.rn.f32x2 %0, %1, t;\n}" : "=l"(r) : "l"(acc), "f"(x), "f"(y));
+  return r;
+}
+__device__ __forceinline__ float sum_f32x2(uint64_t a) {
+  return __uint_as_float((uint32_t)a) + __uint_as_float((uint32_t)(a >> 32));
+}
+__device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
 }
 
+// This lane's J code bytes of a tile (see the tile layout in common.cuh).
 template <int J>
-__device__ __forceinline__ void load_lane_words(const uint8_t* p, uint32_t (&w)[J / 4]) {
+__device__ __forceinline__ void load_tile_words(const uint8_t* tile, int lane, uint32_t (&w)[J / 4]) {
   if constexpr (J == 32) {
-    uint4 a = *reinterpret_cast<const uint4*>(p);
-    uint4 b = *reinterpret_cast<const uint4*>(p + 16);
+    const uint4 a = *reinterpret_cast<const uint4*>(tile + lane * 16);
+    const uint4 b = *reinterpret_cast<const uint4*>(tile + 512 + lane * 16);
     w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w;
     w[4] = b.x; w[5] = b.y; w[6] = b.z; w[7] = b.w;
   } else if constexpr (J == 16) {
-    uint4 a = *reinterpret_cast<const uint4*>(p);
+    const uint4 a = *reinterpret_cast<const uint4*>(tile + lane * 16);
     w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w;
   } else {
-    uint2 a = *reinterpret_cast<const uint2*>(p);
+    const uint2 a = *reinterpret_cast<const uint2*>(tile + lane * 8);
     w[0] = a.x; w[1] = a.y;
   }
 }
 
-// Score of token `lane` of a K tile (lane's J bytes at p).
-template <int J>
-__device__ __forceinline__ float tile_scores(const uint8_t* p, uint32_t lut_lane) {
-  uint32_t w[J / 4];
-  load_lane_words<J>(p, w);
-  float v[J];
-#pragma unroll
-  for (int i = 0; i < J / 4; ++i) {
-    v[4 * i + 0] = lds_f32(code_addr<0>(w[i], lut_lane));
-    v[4 * i + 1] = lds_f32(code_addr<1>(w[i], lut_lane));
-    v[4 * i + 2] = lds_f32(code_addr<2>(w[i], lut_lane));
-    v[4 * i + 3] = lds_f32(code_addr<3>(w[i], lut_lane));
-  }
-#pragma unroll
-  for (int m = J / 2; m >= 1; m >>= 1) {
-#pragma unroll
-    for (int i = 0; i < m; ++i) v[i] += __shfl_xor_sync(0xffffffffu, v[i + m], m);
-  }
-  return v[0];
+// Shared address of the lookup-table entry of code = byte K of w for the
+// lane's column at that step: col holds the region base (bytes 2-3) and the
+// column offset (byte 0); the code becomes byte 1 (row of 256 bytes).
+template <int K>
+__device__ __forceinline__ uint32_t entry_addr(uint32_t w, uint32_t col) {
+  return __byte_perm(w, col, 0x7604u | (K << 4));
 }
 
-// Adds the weights of the group's J tokens into the histogram columns of this
-// lane for one V tile (lane's J bytes at p; weights at qg[0..J)).
+// Scores of this lane's token in two tiles at once (two independent chains
+// for latency hiding): the sum over its J codes of the lookup-table column
+// the rotation assigns to each step.
 template <int J>
-__device__ __forceinline__ void tile_hist(const uint8_t* p, const uint32_t* qg, uint32_t hist_lane) {
-  uint32_t w[J / 4];
-  load_lane_words<J>(p, w);
+__device__ __forceinline__ void token_score2(const uint8_t* t0, const uint8_t* t1, int lane,
+                                             const uint32_t (&col)[J], float& s0, float& s1) {
+  uint32_t w0[J / 4], w1[J / 4];
+  load_tile_words<J>(t0, lane, w0);
+  load_tile_words<J>(t1, lane, w1);
+  uint64_t a01 = 0, a23 = 0, b01 = 0, b23 = 0;   // packed fp32 pairs, 0 bits = (0, 0)
 #pragma unroll
   for (int i = 0; i < J / 4; ++i) {
-    uint4 qq = *reinterpret_cast<const uint4*>(qg + 4 * i);
-    red_add_u32(code_addr<0>(w[i], hist_lane), qq.x);
-    red_add_u32(code_addr<1>(w[i], hist_lane), qq.y);
-    red_add_u32(code_addr<2>(w[i], hist_lane), qq.z);
-    red_add_u32(code_addr<3>(w[i], hist_lane), qq.w);
+    const float x0 = lds_f32(entry_addr<0>(w0[i], col[4 * i + 0]));
+    const float y0 = lds_f32(entry_addr<0>(w1[i], col[4 * i + 0]));
+    const float x1 = lds_f32(entry_addr<1>(w0[i], col[4 * i + 1]));
+    const float y1 = lds_f32(entry_addr<1>(w1[i], col[4 * i + 1]));
+    const float x2 = lds_f32(entry_addr<2>(w0[i], col[4 * i + 2]));
+    const float y2 = lds_f32(entry_addr<2>(w1[i], col[4 * i + 2]));
+    const float x3 = lds_f32(entry_addr<3>(w0[i], col[4 * i + 3]));
+    const float y3 = lds_f32(entry_addr<3>(w1[i], col[4 * i + 3]));
+    a01 = add_f32x2(a01, x0, x1);
+    b01 = add_f32x2(b01, y0, y1);
+    a23 = add_f32x2(a23, x2, x3);
+    b23 = add_f32x2(b23, y2, y3);
+  }
+  s0 = sum_f32x2(a01) + sum_f32x2(a23);
+  s1 = sum_f32x2(b01) + sum_f32x2(b23);
+}
+
+// Adds this lane's token weights of two tiles into the histogram bins of
+// their codes.
+template <int J>
+__device__ __forceinline__ void token_hist2(const uint8_t* t0, const uint8_t* t1, int lane,
+                                            const uint32_t (&col)[J], uint32_t q0, uint32_t q1) {
+  uint32_t w0[J / 4], w1[J / 4];
+  load_tile_words<J>(t0, lane, w0);
+  load_tile_words<J>(t1, lane, w1);
+#pragma unroll
+  for (int i = 0; i < J / 4; ++i) {
+    red_hist_u32(entry_addr<0>(w0[i], col[4 * i + 0]), q0);
+    red_hist_u32(entry_addr<0>(w1[i], col[4 * i + 0]), q1);
+    red_hist_u32(entry_addr<1>(w0[i], col[4 * i + 1]), q0);
+    red_hist_u32(entry_addr<1>(w1[i], col[4 * i + 1]), q1);
+    red_hist_u32(entry_addr<2>(w0[i], col[4 * i + 2]), q0);
+    red_hist_u32(entry_addr<2>(w1[i], col[4 * i + 2]), q1);
+    red_hist_u32(entry_addr<3>(w0[i], col[4 * i + 3]), q0);
+    red_hist_u32(entry_addr<3>(w1[i], col[4 * i + 3]), q1);
   }
 }
 
@@ -150,7 +189,6 @@ __device__ __forceinline__ void tile_hist(const uint8_t* p, const uint32_t* qg, 
 template <int W, typename CBT>
 __device__ __forceinline__ void load_vec(const CBT* p, bool ok, float (&v)[W]) {
   if constexpr (sizeof(CBT) == 2) {
-    static_assert(W % 4 == 0 || W == 2, "bf16 vectors of 2, 4, 8 or 16");
     if constexpr (W == 2) {
       const uint32_t a = ok ? *reinterpret_cast<const uint32_t*>(p) : 0u;
       v[0] = bf16_lo(a); v[1] = bf16_hi(a);
@@ -180,6 +218,38 @@ __device__ __forceinline__ float load_q(const void* q, int q_bf16, size_t i) {
                 : reinterpret_cast<const float*>(q)[i];
 }
 
+// Last-split merge with one global round trip: every split's (o, m, l) row is
+// staged in shared memory (`sm`, `cap` floats), then combined there.  Falls
+// back to the two-phase combine when the rows do not fit.
+__device__ __forceinline__ void combine_staged(const float* part, int n_splits, int D, void* out, int out_bf16,
+                                               float* lse, float* sm, int cap, int tid, int nthr) {
+  const int row = D + 4;
+  if (n_splits * row > cap) {
+    combine_splits(part, n_splits, D, out, out_bf16, lse, sm, tid, nthr, ConsumerSync{});
+    return;
+  }
+  for (int i = tid; i < n_splits * row; i += nthr) sm[i] = __ldcg(part + i);
+  consumer_sync();
+  float M = -INFINITY;
+  for (int s = 0; s < n_splits; ++s) M = fmaxf(M, sm[s * row + D]);
+  float L = 0.f;
+  for (int s = 0; s < n_splits; ++s)
+    if (sm[s * row + D] != -INFINITY) L += sm[s * row + D + 1] * exp2f(sm[s * row + D] - M);
+  if (tid < D) {
+    float o = 0.f;
+    if (M != -INFINITY) {
+      for (int s = 0; s < n_splits; ++s)
+        if (sm[s * row + D] != -INFINITY) o = fmaf(sm[s * row + tid], exp2f(sm[s * row + D] - M), o);
+      o = L > 0.f ? o / L : 0.f;
+    }
+    if (out_bf16)
+      ((__nv_bfloat16*)out)[tid] = __float2bfloat16_rn(o);
+    else
+      ((float*)out)[tid] = o;
+  }
+  if (lse && tid == 0) *lse = (M == -INFINITY || !(L > 0.f)) ? -INFINITY : (M + log2f(L)) * 0.6931471805599453f;
+}
+
 template <int J, int D, typename CBT>
 __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams p) {
   extern __shared__ __align__(1024) uint8_t dyn[];
@@ -188,9 +258,28 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
   const int group = p.Hq / p.H;
   const int h = hq / group;
   constexpr int W = D / J;
+  constexpr int kPer = 256 * J / (kNW * 32);   // lookup-table entries per consumer thread
+
+  // ---- loads that depend only on the block index, all issued up front ----
+  int ctx = __ldg(p.ctx_len + r);
+  const int64_t body_off = __ldg(p.body_off + r);
+  const int64_t win_off = __ldg(p.win_off + r);
+  const size_t unit = (size_t)r * p.Hq + hq;
+  float qj[W];                     // q[j*W .. j*W+W) of this thread's slot j = tid % J
+  float wk[kPer][W];               // B^K_t entries (c, j) = tid + 512k, code-major slice
+  const CBT* bk = reinterpret_cast<const CBT*>(p.cbK_slice) + (size_t)h * p.C * J * W;
+  if (tid < kNW * 32) {
+    const int j = tid % J;
+#pragma unroll
+    for (int w = 0; w < W; ++w) qj[w] = load_q(p.q, p.q_bf16, unit * D + j * W + w) * p.scale_log2;
+#pragma unroll
+    for (int k = 0; k < kPer; ++k) {
+      const int e = tid + k * kNW * 32;
+      load_vec<W>(bk + (size_t)e * W, e / J < p.C, wk[k]);
+    }
+  }
 
   // ---- work of this CTA -------------------------------------------------
-  int ctx = __ldg(p.ctx_len + r);
   bool bad = false;
   if (ctx < 0 || ctx > p.max_ctx) {
     if (tid == 0 && split == 0) set_fault(p.status, LOOPVQ_FAULT_CTX_RANGE);
@@ -201,7 +290,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
   const int has_win = n_win > 0 ? 1 : 0;
   const int n_body_splits = (cs.body + p.split_len - 1) / p.split_len;
   const int n_splits = has_win + n_body_splits;
-  const size_t unit = (size_t)r * p.Hq + hq;
   if (ctx == 0) {  // empty context: zero output, lse -inf
     if (split == 0) {
       for (int d = tid; d < D; d += blockDim.x) {
@@ -215,12 +303,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
   if (split >= n_splits) return;
   const bool is_window = split < has_win;
   const int bsplit = split - has_win;
-  int64_t win_off = 0, body_off = 0;
   if (is_window) {
-    win_off = __ldg(p.win_off + r);
     if (win_off < 0 || win_off + n_win > p.win_pool_tokens) bad = true;
   } else {
-    body_off = __ldg(p.body_off + r);
     if (body_off < 0 || (body_off & 31) || body_off + cs.body > p.body_pool_tokens) bad = true;
   }
   if (bad && tid == 0) set_fault(p.status, LOOPVQ_FAULT_POOL_RANGE);
@@ -228,27 +313,43 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
   const int n_tok = bad ? 0 : (is_window ? n_win : min(p.split_len, cs.body - tok0));
   const int n_tiles = (n_tok + 31) >> 5;
 
-  // ---- shared memory plan ------------------------------------------------
+  // ---- shared memory ------------------------------------------------------
+  // 64 KB-aligned [code][table | histogram] region; misc, scores and ring
+  // stages go below it while they fit, the rest above it.
   const uint32_t sbase = smem_u32(dyn);
-  const uint32_t region = (sbase + (kRegionAlign - 1)) & ~(uint32_t)(kRegionAlign - 1);
-  uint8_t* const dyn_region = dyn + (region - sbase);
-  float* const lut = reinterpret_cast<float*>(dyn_region);                 // [256][32]
-  uint32_t* const hist = reinterpret_cast<uint32_t*>(dyn_region + 32768);  // [256][32]
-  uint8_t* const ring = dyn_region + 65536;
-  float* const sc = reinterpret_cast<float*>(ring + kStages * kStageBytes);
-  uint8_t* const misc = reinterpret_cast<uint8_t*>(sc) + kScoresBytes;
+  const uint32_t region = (sbase + (kRegionBytes - 1)) & ~(uint32_t)(kRegionBytes - 1);
+  uint32_t lo = sbase, hi = region + kRegionBytes;
+  auto place = [&](uint32_t bytes) -> uint32_t {
+    if (lo + bytes <= region) { const uint32_t a = lo; lo += bytes; return a; }
+    const uint32_t a = hi; hi += bytes; return a;
+  };
+  const uint32_t misc_a = place(kMiscBytes);
+  const uint32_t sc_a = place(kScoresBytes);
+  uint32_t stage_a[kStages];
+#pragma unroll
+  for (int i = 0; i < kStages; ++i) stage_a[i] = place(kStageBytes);
+  if (hi > sbase + kDynSmem) {  // cannot happen with the 1 KB reserved window start
+    if (tid == 0) set_fault(p.status, LOOPVQ_FAULT_TIMEOUT);
+    return;
+  }
+  uint8_t* const region_p = dyn + (region - sbase);
+  float* const lut = reinterpret_cast<float*>(region_p);         // row c: lut[c*64 + col]
+  uint32_t* const hist = reinterpret_cast<uint32_t*>(region_p);  // row c: hist[c*64 + 32 + col]
+  auto stage_ptr = [&](int i) -> uint8_t* { return dyn + (stage_a[i] - sbase); };
+  float* const sc = reinterpret_cast<float*>(dyn + (sc_a - sbase));
+  uint8_t* const misc = dyn + (misc_a - sbase);
   uint64_t* const full_bar = reinterpret_cast<uint64_t*>(misc);
   uint64_t* const empty_bar = full_bar + kStages;
-  float* const qs = reinterpret_cast<float*>(misc + 128);         // [D <= 128] scaled query
-  float* const red = reinterpret_cast<float*>(misc + 128 + 512);  // [kNW * 2]
-  uint32_t* const qbuf = reinterpret_cast<uint32_t*>(misc + 1024);  // [kNW][32]
-  int* const flag = reinterpret_cast<int*>(misc + 1024 + kNW * 128);
+  float* const red = reinterpret_cast<float*>(misc + 256);          // [kNW * 2]
+  int* const flag = reinterpret_cast<int*>(misc + 512);
 
-  // chunks: window -> one chunk per 32 tokens (K rows then V rows);
-  //         body   -> K tiles then V tiles, tiles_per_chunk each.
+  // chunks: window -> K rows then V rows, kRowsPerChunk tokens each;
+  //         body   -> K tiles then V tiles, kTilesPerChunk each.
   constexpr int kTilesPerChunk = kStageBytes / (32 * J);
-  const int n_chunks_half = is_window ? (n_tok + 31) / 32 : (n_tiles + kTilesPerChunk - 1) / kTilesPerChunk;
-  const int n_chunks = is_window ? n_chunks_half : 2 * n_chunks_half;
+  constexpr int kRowsPerChunk = kStageBytes / (D * 2);
+  const int n_chunks_half = is_window ? (n_tok + kRowsPerChunk - 1) / kRowsPerChunk
+                                      : (n_tiles + kTilesPerChunk - 1) / kTilesPerChunk;
+  const int n_chunks = 2 * n_chunks_half;
 
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -262,6 +363,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
   // ======================= producer warp ===================================
   if (warp == kNW) {
     if (lane == 0) {
+      if (!is_window && n_tok > 0)  // the epilogue's codebook slice: warm L2 now
+        prefetch_l2(reinterpret_cast<const CBT*>(p.cbV_slice) + (size_t)h * p.C * D, (uint32_t)(p.C * D * sizeof(CBT)));
       for (int k = 0; k < n_chunks; ++k) {
         const int s = k % kStages;
         if (k >= kStages) {
@@ -270,16 +373,16 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
             break;
           }
         }
-        const uint32_t dst = smem_u32(ring + s * kStageBytes);
+        const uint32_t dst = stage_a[s];
         const uint32_t fb = smem_u32(full_bar + s);
         if (is_window) {
-          const int t0 = k * 32;
-          const int nt = min(32, n_tok - t0);
+          const bool vpass = k >= n_chunks_half;
+          const int t0 = (vpass ? k - n_chunks_half : k) * kRowsPerChunk;
+          const int nt = min(kRowsPerChunk, n_tok - t0);
           const uint32_t bytes = (uint32_t)nt * D * 2;
           const size_t row0 = ((size_t)h * p.win_pool_tokens + win_off + t0) * D;
-          mbar_arrive_expect_tx(fb, 2 * bytes);
-          bulk_g2s(dst, p.winK + row0, bytes, fb);
-          bulk_g2s(dst + 32 * D * 2, p.winV + row0, bytes, fb);
+          mbar_arrive_expect_tx(fb, bytes);
+          bulk_g2s(dst, (vpass ? p.winV : p.winK) + row0, bytes, fb);
         } else {
           const bool vpass = k >= n_chunks_half;
           const int c = vpass ? k - n_chunks_half : k;
@@ -300,125 +403,146 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
   float* const part = p.partials + (unit * p.max_splits + split) * (size_t)(D + 4);
   const int ctid = tid;  // 0 .. kNW*32-1
 
-  // scaled query (log2 units)
-  for (int d = ctid; d < D; d += kNW * 32) qs[d] = load_q(p.q, p.q_bf16, unit * D + d) * p.scale_log2;
-  consumer_sync();
-
   if (is_window) {
-    // lane owns channels lane*CPL .. lane*CPL+CPL-1 (CPL = D/32 = 2 or 4)
+    // Two passes over the bf16 rows: scores of every window token (lanes own
+    // channels lane*CPL.., four tokens per warp in flight), the window max,
+    // then the weighted sum of the value rows.
     constexpr int CPL = D >> 5;
-    float qv[4], ov[4] = {0.f, 0.f, 0.f, 0.f};
+    float qv[CPL], ov[CPL];
 #pragma unroll
-    for (int i = 0; i < CPL; ++i) qv[i] = qs[lane * CPL + i];
-    float m = -INFINITY, l = 0.f;
-    for (int k = 0; k < n_chunks; ++k) {
+    for (int i = 0; i < CPL; ++i) {
+      qv[i] = load_q(p.q, p.q_bf16, unit * D + lane * CPL + i) * p.scale_log2;
+      ov[i] = 0.f;
+    }
+    float mx = -INFINITY;
+    for (int k = 0; k < n_chunks_half; ++k) {
       const int s = k % kStages;
       if (!mbar_wait_bounded(smem_u32(full_bar + s), (k / kStages) & 1)) set_fault(p.status, LOOPVQ_FAULT_TIMEOUT);
-      const uint8_t* st = ring + s * kStageBytes;
-      const int nt = min(32, n_tok - k * 32);
-      for (int tkn = warp; tkn < nt; tkn += kNW) {
-        const uint8_t* kr = st + (size_t)tkn * D * 2 + lane * CPL * 2;
-        const uint8_t* vr = st + 32 * D * 2 + (size_t)tkn * D * 2 + lane * CPL * 2;
-        float kf[4], vf[4];
-        if constexpr (CPL == 4) {
-          uint2 a = *reinterpret_cast<const uint2*>(kr);
-          uint2 b = *reinterpret_cast<const uint2*>(vr);
-          kf[0] = bf16_lo(a.x); kf[1] = bf16_hi(a.x); kf[2] = bf16_lo(a.y); kf[3] = bf16_hi(a.y);
-          vf[0] = bf16_lo(b.x); vf[1] = bf16_hi(b.x); vf[2] = bf16_lo(b.y); vf[3] = bf16_hi(b.y);
-        } else {
-          uint32_t a = *reinterpret_cast<const uint32_t*>(kr);
-          uint32_t b = *reinterpret_cast<const uint32_t*>(vr);
-          kf[0] = bf16_lo(a); kf[1] = bf16_hi(a); kf[2] = kf[3] = 0.f;
-          vf[0] = bf16_lo(b); vf[1] = bf16_hi(b); vf[2] = vf[3] = 0.f;
+      const uint8_t* st = stage_ptr(s);
+      const int nt = min(kRowsPerChunk, n_tok - k * kRowsPerChunk);
+      for (int b0 = warp; b0 < nt; b0 += 4 * kNW) {
+        float dot[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int tkn = b0 + u * kNW < nt ? b0 + u * kNW : b0;
+          const uint8_t* kr = st + (size_t)tkn * D * 2 + lane * CPL * 2;
+          float kf[CPL];
+          if constexpr (CPL == 4) {
+            const uint2 a = *reinterpret_cast<const uint2*>(kr);
+            kf[0] = bf16_lo(a.x); kf[1] = bf16_hi(a.x); kf[2] = bf16_lo(a.y); kf[3] = bf16_hi(a.y);
+          } else {
+            const uint32_t a = *reinterpret_cast<const uint32_t*>(kr);
+            kf[0] = bf16_lo(a); kf[1] = bf16_hi(a);
+          }
+          dot[u] = 0.f;
+#pragma unroll
+          for (int i = 0; i < CPL; ++i) dot[u] = fmaf(qv[i], kf[i], dot[u]);
         }
-        float sdot = 0.f;
 #pragma unroll
-        for (int i = 0; i < CPL; ++i) sdot = fmaf(qv[i], kf[i], sdot);
+        for (int o = 16; o >= 1; o >>= 1) {
 #pragma unroll
-        for (int o = 16; o >= 1; o >>= 1) sdot += __shfl_xor_sync(0xffffffffu, sdot, o);
-        if (sdot > m) {
-          const float corr = exp2f(m - sdot);
-          l *= corr;
-#pragma unroll
-          for (int i = 0; i < 4; ++i) ov[i] *= corr;
-          m = sdot;
+          for (int u = 0; u < 4; ++u) dot[u] += __shfl_xor_sync(0xffffffffu, dot[u], o);
         }
-        const float pw = exp2f(sdot - m);
-        l += pw;
 #pragma unroll
-        for (int i = 0; i < CPL; ++i) ov[i] = fmaf(pw, vf[i], ov[i]);
+        for (int u = 0; u < 4; ++u) {
+          const int tkn = b0 + u * kNW;
+          if (tkn < nt) {
+            if (lane == u) sc[k * kRowsPerChunk + tkn] = dot[u];
+            mx = fmaxf(mx, dot[u]);
+          }
+        }
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(empty_bar + s));
     }
-    // merge the warps' (m, l, o): reuse the score buffer as [kNW][D + 2]
-    float* wpart = sc;
-#pragma unroll
-    for (int i = 0; i < CPL; ++i) wpart[warp * (D + 2) + lane * CPL + i] = ov[i];
-    if (lane == 0) {
-      wpart[warp * (D + 2) + D] = m;
-      wpart[warp * (D + 2) + D + 1] = l;
-    }
+    if (lane == 0) red[warp] = mx;
     consumer_sync();
-    float M = -INFINITY;
-    for (int w = 0; w < kNW; ++w) M = fmaxf(M, wpart[w * (D + 2) + D]);
-    for (int d = ctid; d < D + 2; d += kNW * 32) {
-      float acc = 0.f;
-      if (d < D || d == D + 1) {
-        for (int w = 0; w < kNW; ++w) {
-          const float mw = wpart[w * (D + 2) + D];
-          if (mw != -INFINITY) acc += wpart[w * (D + 2) + d] * exp2f(mw - M);
+    float m = -INFINITY;
+    for (int w = 0; w < kNW; ++w) m = fmaxf(m, red[w]);
+    float l = 0.f;
+    for (int k = n_chunks_half; k < n_chunks; ++k) {
+      const int s = k % kStages;
+      if (!mbar_wait_bounded(smem_u32(full_bar + s), (k / kStages) & 1)) set_fault(p.status, LOOPVQ_FAULT_TIMEOUT);
+      const uint8_t* st = stage_ptr(s);
+      const int kv = k - n_chunks_half;
+      const int nt = min(kRowsPerChunk, n_tok - kv * kRowsPerChunk);
+      for (int tkn = warp; tkn < nt; tkn += kNW) {
+        const float pw = exp2f(sc[kv * kRowsPerChunk + tkn] - m);
+        const uint8_t* vr = st + (size_t)tkn * D * 2 + lane * CPL * 2;
+        l += pw;
+        if constexpr (CPL == 4) {
+          const uint2 b = *reinterpret_cast<const uint2*>(vr);
+          ov[0] = fmaf(pw, bf16_lo(b.x), ov[0]); ov[1] = fmaf(pw, bf16_hi(b.x), ov[1]);
+          ov[2] = fmaf(pw, bf16_lo(b.y), ov[2]); ov[3] = fmaf(pw, bf16_hi(b.y), ov[3]);
+        } else {
+          const uint32_t b = *reinterpret_cast<const uint32_t*>(vr);
+          ov[0] = fmaf(pw, bf16_lo(b), ov[0]); ov[1] = fmaf(pw, bf16_hi(b), ov[1]);
         }
       }
-      part[d] = (d == D) ? M : acc;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(empty_bar + s));
+    }
+    // every warp used the same max: the merge is a plain sum
+    consumer_sync();  // all score reads done before the buffer is reused
+    float* wpart = sc;  // [kNW][D + 1]
+#pragma unroll
+    for (int i = 0; i < CPL; ++i) wpart[warp * (D + 1) + lane * CPL + i] = ov[i];
+    if (lane == 0) wpart[warp * (D + 1) + D] = l;
+    consumer_sync();
+    for (int d = ctid; d < D + 2; d += kNW * 32) {
+      float acc = 0.f;
+      if (d != D) {
+        const int dd = d == D + 1 ? D : d;
+        for (int w = 0; w < kNW; ++w) acc += wpart[w * (D + 1) + dd];
+      }
+      part[d] = (d == D) ? m : acc;
     }
   } else {
-    // ---- LUT of step t: LUT[c][g*J + j] = sum_w qs[j*W+w] * B^K_t[c][j][w].
-    // Entry e = (c, j) is one W-vector of the code-major slice; a thread owns
-    // entries ctid + 512k, all loads issued before any use.
-    const CBT* bk = reinterpret_cast<const CBT*>(p.cbK_slice) + (size_t)h * p.C * J * W;
+    // ---- LUT of step t: LUT[c][g*J + j] = sum_w q_{j*W+w} * B^K_t[c][j][w]
     {
-      constexpr int kPer = 256 * J / (kNW * 32);
-      float wv[kPer][W];
+      const int j = ctid % J;
 #pragma unroll
       for (int k = 0; k < kPer; ++k) {
-        const int e = ctid + k * kNW * 32;
-        const int c = e / J;
-        load_vec<W>(bk + (size_t)e * W, c < p.C, wv[k]);
-      }
-#pragma unroll
-      for (int k = 0; k < kPer; ++k) {
-        const int e = ctid + k * kNW * 32;
-        const int c = e / J, j = e % J;
+        const int c = (ctid + k * kNW * 32) / J;
         float acc = 0.f;
 #pragma unroll
-        for (int w = 0; w < W; ++w) acc = fmaf(qs[j * W + w], wv[k][w], acc);
+        for (int w = 0; w < W; ++w) acc = fmaf(qj[w], wk[k][w], acc);
         if (c >= p.C) acc = __int_as_float(0x7fc00000);  // NaN marks a code >= n_codes
 #pragma unroll
-        for (int g = 0; g < 32 / J; ++g) lut[c * 32 + g * J + j] = acc;
+        for (int g = 0; g < 32 / J; ++g) lut[c * 64 + g * J + j] = acc;
       }
     }
-    for (int e = ctid; e < 256 * 32; e += kNW * 32) hist[e] = 0u;
+    for (int e = ctid; e < 256 * 32; e += kNW * 32) hist[(e >> 5) * 64 + 32 + (e & 31)] = 0u;
+    // this lane's column at step s: (lane / J) * J + (s + lane) mod J
+    uint32_t col[J];
+#pragma unroll
+    for (int s = 0; s < J; ++s) col[s] = region | (uint32_t)(((lane / J) * J + ((s + lane) % J)) * 4);
     consumer_sync();
 
-    const uint32_t lut_lane = region + lane * 4;
-    const uint32_t hist_lane = region + 32768 + lane * 4;
     // ---- pass K: scores and split maximum
     float mx = -INFINITY;
     bool nan_seen = false;
     for (int k = 0; k < n_chunks_half; ++k) {
       const int s = k % kStages;
       if (!mbar_wait_bounded(smem_u32(full_bar + s), (k / kStages) & 1)) set_fault(p.status, LOOPVQ_FAULT_TIMEOUT);
-      const uint8_t* st = ring + s * kStageBytes;
+      const uint8_t* st = stage_ptr(s);
       const int nt = min(kTilesPerChunk, n_tiles - k * kTilesPerChunk);
-      for (int tl = warp; tl < nt; tl += kNW) {
-        const float sv = tile_scores<J>(st + tl * 32 * J + lane * J, lut_lane);
-        const int tok = (k * kTilesPerChunk + tl) * 32 + lane;
-        const bool valid = tok < n_tok;
-        if (valid && sv != sv) nan_seen = true;
-        const float s2 = valid ? sv : -INFINITY;
-        sc[tok] = s2;
-        mx = fmaxf(mx, s2);
+      for (int tl = warp; tl < nt; tl += 2 * kNW) {
+        const int tl2 = tl + kNW < nt ? tl + kNW : tl;
+        float sv0, sv1;
+        token_score2<J>(st + tl * 32 * J, st + tl2 * 32 * J, lane, col, sv0, sv1);
+        const int tok0c = (k * kTilesPerChunk + tl) * 32 + lane;
+        const bool v0 = tok0c < n_tok;
+        if (v0 && sv0 != sv0) nan_seen = true;
+        sc[tok0c] = v0 ? sv0 : -INFINITY;
+        mx = fmaxf(mx, v0 ? sv0 : -INFINITY);
+        if (tl2 != tl) {
+          const int tok1c = (k * kTilesPerChunk + tl2) * 32 + lane;
+          const bool v1 = tok1c < n_tok;
+          if (v1 && sv1 != sv1) nan_seen = true;
+          sc[tok1c] = v1 ? sv1 : -INFINITY;
+          mx = fmaxf(mx, v1 ? sv1 : -INFINITY);
+        }
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(empty_bar + s));
@@ -430,36 +554,45 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
     consumer_sync();
     float m = -INFINITY;
     for (int w = 0; w < kNW; ++w) m = fmaxf(m, red[w]);
-    // fixed-point scale: n_tok * 2^S < 2^32
-    const int S = 31 - (31 - __clz(max(n_tok, 1)));
+    // fixed-point scale: n_tok * 2^S < 2^32 with S = clz(n_tok)
+    const int S = __clz(max(n_tok, 1));
     const float scaleS = exp2f((float)S);
 
     // ---- pass V: weights into the histogram
     uint32_t qsum = 0;
-    uint32_t* const qw = qbuf + warp * 32;
-    const int g0 = (lane / J) * J;
     for (int k = n_chunks_half; k < n_chunks; ++k) {
       const int s = k % kStages;
       if (!mbar_wait_bounded(smem_u32(full_bar + s), (k / kStages) & 1)) set_fault(p.status, LOOPVQ_FAULT_TIMEOUT);
-      const uint8_t* st = ring + s * kStageBytes;
+      const uint8_t* st = stage_ptr(s);
       const int kv = k - n_chunks_half;
       const int nt = min(kTilesPerChunk, n_tiles - kv * kTilesPerChunk);
-      for (int tl = warp; tl < nt; tl += kNW) {
-        const int tok = (kv * kTilesPerChunk + tl) * 32 + lane;
-        uint32_t qv = 0;
-        if (tok < n_tok) {
-          const float pw = exp2f(sc[tok] - m);
-          const uint32_t seq = (uint32_t)(body_off + tok0 + tok);
-          const float u = (float)((seq * 2654435769u) >> 8) * (1.0f / 16777216.0f);
-          qv = __float2uint_rd(fmaf(pw, scaleS, u));
+      for (int tl = warp; tl < nt; tl += 2 * kNW) {
+        const int tl2 = tl + kNW < nt ? tl + kNW : tl;
+        uint32_t qv[2];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const int tok = (kv * kTilesPerChunk + (u ? tl2 : tl)) * 32 + lane;
+          qv[u] = 0;
+          if (tok < n_tok && (u == 0 || tl2 != tl)) {
+            const float pw = exp2f(sc[tok] - m);
+            const uint32_t seq = (uint32_t)(body_off + tok0 + tok);
+            const float uu = (float)((seq * 2654435769u) >> 8) * (1.0f / 16777216.0f);
+            qv[u] = __float2uint_rd(fmaf(pw, scaleS, uu));
+          }
+          qsum += qv[u];
         }
-        qsum += qv;
-        qw[lane] = qv;
-        __syncwarp();
-        tile_hist<J>(st + tl * 32 * J + lane * J, qw + g0, hist_lane);
-        __syncwarp();
+        token_hist2<J>(st + tl * 32 * J, st + tl2 * 32 * J, lane, col, qv[0], qv[1]);
       }
+      __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(empty_bar + s));
+    }
+    // epilogue operands: entries (c, j) = ctid + 512k of the code-major V slice
+    const CBT* bv = reinterpret_cast<const CBT*>(p.cbV_slice) + (size_t)h * p.C * D;
+    float vv[kPer][W];
+#pragma unroll
+    for (int k = 0; k < kPer; ++k) {
+      const int e = ctid + k * kNW * 32;
+      load_vec<W>(bv + (size_t)e * W, e / J < p.C, vv[k]);
     }
 #pragma unroll
     for (int o = 16; o >= 1; o >>= 1) qsum += __shfl_xor_sync(0xffffffffu, qsum, o);
@@ -467,19 +600,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
     consumer_sync();
 
     // ---- epilogue: o[d] = 2^-S sum_c hist[j][c] B^V_t[c][j][w].  Thread
-    // ctid owns entries e = (c, j) = ctid + 512k and accumulates its W
-    // outputs over them; the 512/J partial groups per output are summed
-    // through shared memory (the LUT region is free by now).
-    const CBT* bv = reinterpret_cast<const CBT*>(p.cbV_slice) + (size_t)h * p.C * D;
+    // ctid accumulates its W outputs over entries (c, j) = ctid + 512k; the
+    // 512/J partial groups per output are summed through shared memory (the
+    // LUT region is free by now).
     {
-      constexpr int kPer = 256 * J / (kNW * 32);
       constexpr int kGroups = (kNW * 32) / J;
-      float vv[kPer][W];
-#pragma unroll
-      for (int k = 0; k < kPer; ++k) {
-        const int e = ctid + k * kNW * 32;
-        load_vec<W>(bv + (size_t)e * W, e / J < p.C, vv[k]);
-      }
       float acc[W];
 #pragma unroll
       for (int w = 0; w < W; ++w) acc[w] = 0.f;
@@ -489,7 +614,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
         const int c = (ctid + k * kNW * 32) / J;
         uint32_t hs = 0;
 #pragma unroll
-        for (int g = 0; g < 32 / J; ++g) hs += hist[c * 32 + g * J + j];
+        for (int g = 0; g < 32 / J; ++g) hs += hist[c * 64 + 32 + g * J + j];
         if (c < p.C) {
           const float hf = (float)hs;
 #pragma unroll
@@ -499,10 +624,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
       // bins of codes >= n_codes must be empty
       if (p.C < 256) {
         bool any = false;
-        for (int e = p.C * 32 + ctid; e < 256 * 32; e += kNW * 32) any |= hist[e] != 0u;
+        for (int e = p.C * 32 + ctid; e < 256 * 32; e += kNW * 32) any |= hist[(e >> 5) * 64 + 32 + (e & 31)] != 0u;
         if (any) set_fault(p.status, LOOPVQ_FAULT_CODE_RANGE);
       }
-      float* ored = lut;  // [kGroups][D]
+      float* ored = reinterpret_cast<float*>(stage_ptr(0));  // [kGroups][D]; the ring is drained
       const int grp = ctid / J;
 #pragma unroll
       for (int w = 0; w < W; ++w) ored[grp * D + j * W + w] = acc[w];
@@ -523,19 +648,21 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
   }
 
   // ---- split ticket and combine -------------------------------------------
-  __threadfence();
   consumer_sync();
   if (ctid == 0) {
+    __threadfence();
     const uint32_t t = atomicAdd(p.tickets + unit, 1u);
+    __threadfence();
     *flag = (t == (uint32_t)(n_splits - 1)) ? 1 : 0;
   }
   consumer_sync();
   if (*flag) {
-    __threadfence();
-    combine_splits(p.partials + unit * p.max_splits * (size_t)(D + 4), n_splits, D,
+    // the drained ring (stage 1) is the combine scratch
+    combine_staged(p.partials + unit * p.max_splits * (size_t)(D + 4), n_splits, D,
                    p.out_bf16 ? (void*)(reinterpret_cast<__nv_bfloat16*>(p.out) + unit * D)
                               : (void*)(reinterpret_cast<float*>(p.out) + unit * D),
-                   p.out_bf16, p.lse ? p.lse + unit : nullptr);
+                   p.out_bf16, p.lse ? p.lse + unit : nullptr, reinterpret_cast<float*>(stage_ptr(1)),
+                   kStageBytes / 4, ctid, kNW * 32);
     if (ctid == 0) atomicExch(p.tickets + unit, 0u);
   }
 }
@@ -621,7 +748,7 @@ extern "C" loopvq_status loopvq_decode_attn(const loopvq_codebook_desc* desc, co
 
   const int64_t units = (int64_t)layout->batch * g.Hq;
   const DecodePlan pl = decode_plan(units, max_body_tokens(layout), device_sm_count());
-  if (units > 65535LL * 65535LL || pl.max_splits > 1 << 20 || layout->batch > 65535 || g.Hq > 65535)
+  if (units > 65535LL * 65535LL || pl.max_splits > kMaxCombineSplits || layout->batch > 65535 || g.Hq > 65535)
     return LOOPVQ_ERR_UNSUPPORTED;
 
   DecodeParams p;
@@ -751,7 +878,7 @@ extern "C" loopvq_status loopvq_decode_attn_noalloc(const loopvq_codebook_desc* 
   if (ws.total > kLoopvqStaticScratchBytes) return LOOPVQ_ERR_WORKSPACE_TOO_SMALL;
   const int64_t units = (int64_t)layout->batch * g.Hq;
   const DecodePlan pl = decode_plan(units, max_body_tokens(layout), device_sm_count());
-  if (units > 65535LL * 65535LL || pl.max_splits > 1 << 20 || layout->batch > 65535 || g.Hq > 65535)
+  if (units > 65535LL * 65535LL || pl.max_splits > kMaxCombineSplits || layout->batch > 65535 || g.Hq > 65535)
     return LOOPVQ_ERR_UNSUPPORTED;
 
   void* scratch = nullptr;

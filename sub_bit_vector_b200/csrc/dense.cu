@@ -34,6 +34,7 @@ struct DenseParams {
 template <int CPL>  // channels per lane: D / 32
 __global__ void __launch_bounds__(kDThreads) dense_decode_kernel(const DenseParams p) {
   __shared__ float wpart[kDW][CPL * 32 + 2];
+  __shared__ float csm[2 * kMaxCombineSplits + kDThreads];
   __shared__ int flag;
   constexpr int D = CPL * 32;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -148,7 +149,7 @@ __global__ void __launch_bounds__(kDThreads) dense_decode_kernel(const DensePara
   if (flag) {
     __threadfence();
     combine_splits(p.partials + unit * p.max_splits * (size_t)(D + 4), n_splits, D, p.out + unit * D, 0,
-                   p.lse ? p.lse + unit : nullptr);
+                   p.lse ? p.lse + unit : nullptr, csm, tid, kDThreads, BlockSync{});
     if (tid == 0) atomicExch(p.tickets + unit, 0u);
   }
 }
@@ -196,6 +197,7 @@ extern "C" loopvq_status loopvq_dense_decode_attn(int32_t batch, int32_t n_heads
   DenseParams p;
   int len, ms;
   dense_plan(units, max_ctx_len, device_sm_count(), &len, &ms);
+  if (ms > kMaxCombineSplits) return LOOPVQ_ERR_UNSUPPORTED;
   const WsLayout ws = ws_layout(units, ms, head_dim);
   p.H = n_heads_kv; p.Hq = n_heads_q; p.D = head_dim; p.max_ctx = max_ctx_len;
   p.split_len = len; p.max_splits = ms;
