@@ -93,6 +93,17 @@ typedef struct {
 } loopvq_codebook_desc;
 
 /*
+ * Layout flag: the caller guarantees that no kernel that may still be running
+ * when the decode kernel starts writes the layout arrays (ctx_len, body_off,
+ * win_off), the index pools or the codebooks.  The decode kernel is always
+ * launched as a programmatic dependent of the previous kernel in the stream;
+ * with this flag it starts streaming index tiles before that kernel has
+ * finished (queries, windows, outputs and the workspace are still touched
+ * only after it has).  Without the flag nothing is read before then.
+ */
+#define LOOPVQ_LAYOUT_STATIC_INPUTS 0x1u
+
+/*
  * Cache layout of one decode batch.  Request r has ctx_len[r] tokens, the
  * current one included.  They split (project page, "Serving in SGLang") into
  *   sink   = min(ctx, n_sink) first tokens, bf16;
@@ -109,7 +120,7 @@ typedef struct {
   int32_t n_recent;           /* >= 0 (256 on the pages) */
   int32_t page;               /* >= 1 (8 on the pages) */
   int32_t max_ctx_len;        /* host-side bound on every ctx_len[r]; sizes the launch */
-  int32_t reserved;
+  uint32_t flags;             /* LOOPVQ_LAYOUT_* bits, 0 for none */
   const int32_t* ctx_len;     /* device [batch] */
   const int64_t* body_off;    /* device [batch], multiple of 32 */
   const int64_t* win_off;     /* device [batch] */

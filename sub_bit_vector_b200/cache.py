@@ -28,7 +28,8 @@ class DecodeCache:
 
     def __init__(self, *, n_loop, tc, n_heads_kv, head_dim, group_elems, ctx_lens, n_sink=64, n_recent=256,
                  page=8, n_codes=256, n_heads_q=None, cb_dtype=torch.bfloat16, q_dtype=torch.bfloat16,
-                 out_dtype=torch.float32, device="cuda", max_ctx_len=None, pool_slack_tokens=0):
+                 out_dtype=torch.float32, device="cuda", max_ctx_len=None, pool_slack_tokens=0,
+                 static_inputs=False):
         self.device = torch.device(device)
         self.T, self.Tc, self.H, self.D, self.G = n_loop, tc, n_heads_kv, head_dim, group_elems
         self.Hq = n_heads_q or n_heads_kv
@@ -70,9 +71,12 @@ class DecodeCache:
         self.ctx_dev = torch.tensor(self.ctx_lens, dtype=torch.int32, device=dev)
         self.body_off_dev = torch.tensor(body_off, dtype=torch.int64, device=dev)
         self.win_off_dev = torch.tensor(win_off, dtype=torch.int64, device=dev)
+        # static_inputs: this cache's layout arrays, pools and codebooks are not
+        # written by kernels that may still run when a decode starts
         self.layout = L.make_layout(self.batch, n_sink, n_recent, page, self.max_ctx_len, self.ctx_dev,
                                     self.body_off_dev, self.win_off_dev, self.body_pool_tokens,
-                                    self.win_pool_tokens)
+                                    self.win_pool_tokens,
+                                    L.LOOPVQ_LAYOUT_STATIC_INPUTS if static_inputs else 0)
         ws = L.loopvq_decode_workspace_bytes(self.desc, self.layout)
         if ws == 0:
             raise ValueError("invalid cache layout")

@@ -78,7 +78,16 @@ struct DecodeParams {
   float* partials;
   int split_len;   // body tokens per split (multiple of 32, <= kSplitCap)
   int max_splits;  // grid.x
+  int static_inputs;  // layout arrays, index pools and codebooks are not being written by earlier kernels
 };
+
+// Programmatic dependent launch: the kernel is launched so that it may start
+// while the previous kernel in the stream finishes.  Everything that kernel
+// may write (queries, windows, outputs, workspace, and -- unless the caller
+// vouches for them -- layout arrays and index pools) is touched only after
+// griddep_wait().  Codebooks are always treated as constant.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
 __device__ __forceinline__ void consumer_sync() {
   asm volatile("bar.sync 1, %0;" ::"n"(kNW * 32) : "memory");
@@ -260,18 +269,17 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
   constexpr int W = D / J;
   constexpr int kPer = 256 * J / (kNW * 32);   // lookup-table entries per consumer thread
 
+  griddep_launch_dependents();
+  if (!p.static_inputs) griddep_wait();
+
   // ---- loads that depend only on the block index, all issued up front ----
   int ctx = __ldg(p.ctx_len + r);
   const int64_t body_off = __ldg(p.body_off + r);
   const int64_t win_off = __ldg(p.win_off + r);
   const size_t unit = (size_t)r * p.Hq + hq;
-  float qj[W];                     // q[j*W .. j*W+W) of this thread's slot j = tid % J
   float wk[kPer][W];               // B^K_t entries (c, j) = tid + 512k, code-major slice
   const CBT* bk = reinterpret_cast<const CBT*>(p.cbK_slice) + (size_t)h * p.C * J * W;
   if (tid < kNW * 32) {
-    const int j = tid % J;
-#pragma unroll
-    for (int w = 0; w < W; ++w) qj[w] = load_q(p.q, p.q_bf16, unit * D + j * W + w) * p.scale_log2;
 #pragma unroll
     for (int k = 0; k < kPer; ++k) {
       const int e = tid + k * kNW * 32;
@@ -292,6 +300,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
   const int n_splits = has_win + n_body_splits;
   if (ctx == 0) {  // empty context: zero output, lse -inf
     if (split == 0) {
+      griddep_wait();
       for (int d = tid; d < D; d += blockDim.x) {
         if (p.out_bf16) reinterpret_cast<__nv_bfloat16*>(p.out)[unit * D + d] = __float2bfloat16_rn(0.f);
         else reinterpret_cast<float*>(p.out)[unit * D + d] = 0.f;
@@ -363,9 +372,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
   // ======================= producer warp ===================================
   if (warp == kNW) {
     if (lane == 0) {
-      if (!is_window && n_tok > 0)  // the epilogue's codebook slice: warm L2 now
-        prefetch_l2(reinterpret_cast<const CBT*>(p.cbV_slice) + (size_t)h * p.C * D, (uint32_t)(p.C * D * sizeof(CBT)));
-      for (int k = 0; k < n_chunks; ++k) {
+      const uint8_t* vslice = reinterpret_cast<const uint8_t*>(p.cbV_slice) + (size_t)h * p.C * D * sizeof(CBT);
+      const uint32_t vslice_bytes = (uint32_t)(p.C * D * sizeof(CBT));
+      if (!is_window && n_tok > 0) prefetch_l2(vslice, vslice_bytes);  // the epilogue's codebook slice
+      if (is_window && p.static_inputs) griddep_wait();  // window rows may come from the previous kernel
+      const int n_slice = (is_window || n_tok == 0) ? 0 : (int)((vslice_bytes + kStageBytes - 1) / kStageBytes);
+      for (int k = 0; k < n_chunks + n_slice; ++k) {
         const int s = k % kStages;
         if (k >= kStages) {
           if (!mbar_wait_bounded(smem_u32(empty_bar + s), ((k / kStages) - 1) & 1)) {
@@ -375,7 +387,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
         }
         const uint32_t dst = stage_a[s];
         const uint32_t fb = smem_u32(full_bar + s);
-        if (is_window) {
+        if (k >= n_chunks) {  // a piece of the value codebook slice, for the epilogue
+          const uint32_t off = (uint32_t)(k - n_chunks) * kStageBytes;
+          const uint32_t bytes = min((uint32_t)kStageBytes, vslice_bytes - off);
+          mbar_arrive_expect_tx(fb, bytes);
+          bulk_g2s(dst, vslice + off, bytes, fb);
+        } else if (is_window) {
           const bool vpass = k >= n_chunks_half;
           const int t0 = (vpass ? k - n_chunks_half : k) * kRowsPerChunk;
           const int nt = min(kRowsPerChunk, n_tok - t0);
@@ -400,6 +417,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
   }
 
   // ======================= consumer warps ==================================
+  if (p.static_inputs) griddep_wait();  // queries, windows, workspace and outputs from here on
   float* const part = p.partials + (unit * p.max_splits + split) * (size_t)(D + 4);
   const int ctid = tid;  // 0 .. kNW*32-1
 
@@ -501,6 +519,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
     // ---- LUT of step t: LUT[c][g*J + j] = sum_w q_{j*W+w} * B^K_t[c][j][w]
     {
       const int j = ctid % J;
+      float qj[W];                 // q[j*W .. j*W+W) of this thread's slot j, log2 units
+#pragma unroll
+      for (int w = 0; w < W; ++w) qj[w] = load_q(p.q, p.q_bf16, unit * D + j * W + w) * p.scale_log2;
 #pragma unroll
       for (int k = 0; k < kPer; ++k) {
         const int c = (ctid + k * kNW * 32) / J;
@@ -586,13 +607,22 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(empty_bar + s));
     }
-    // epilogue operands: entries (c, j) = ctid + 512k of the code-major V slice
-    const CBT* bv = reinterpret_cast<const CBT*>(p.cbV_slice) + (size_t)h * p.C * D;
+    // epilogue operands: entries (c, j) = ctid + 512k of the code-major value
+    // slice, which the producer bulk-copied into the drained ring stages
+    const int n_slice = (n_tok == 0) ? 0 : (int)((p.C * D * sizeof(CBT) + kStageBytes - 1) / kStageBytes);
+    for (int i = 0; i < n_slice; ++i) {
+      const int k = n_chunks + i;
+      if (!mbar_wait_bounded(smem_u32(full_bar + (k % kStages)), (k / kStages) & 1))
+        set_fault(p.status, LOOPVQ_FAULT_TIMEOUT);
+    }
     float vv[kPer][W];
 #pragma unroll
     for (int k = 0; k < kPer; ++k) {
       const int e = ctid + k * kNW * 32;
-      load_vec<W>(bv + (size_t)e * W, e / J < p.C, vv[k]);
+      const uint32_t off = (uint32_t)e * W * sizeof(CBT);
+      const CBT* src = reinterpret_cast<const CBT*>(stage_ptr((n_chunks + (int)(off / kStageBytes)) % kStages) +
+                                                    off % kStageBytes);
+      load_vec<W>(src, n_slice > 0 && e / J < p.C, vv[k]);
     }
 #pragma unroll
     for (int o = 16; o >= 1; o >>= 1) qsum += __shfl_xor_sync(0xffffffffu, qsum, o);
@@ -615,7 +645,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
         uint32_t hs = 0;
 #pragma unroll
         for (int g = 0; g < 32 / J; ++g) hs += hist[c * 64 + 32 + g * J + j];
-        if (c < p.C) {
+        if (c < p.C && hs != 0u) {
           const float hf = (float)hs;
 #pragma unroll
           for (int w = 0; w < W; ++w) acc[w] = fmaf(hf, vv[k][w], acc[w]);
@@ -627,15 +657,22 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
         for (int e = p.C * 32 + ctid; e < 256 * 32; e += kNW * 32) any |= hist[(e >> 5) * 64 + 32 + (e & 31)] != 0u;
         if (any) set_fault(p.status, LOOPVQ_FAULT_CODE_RANGE);
       }
-      float* ored = reinterpret_cast<float*>(stage_ptr(0));  // [kGroups][D]; the ring is drained
+      // [kGroups][D] partial sums in the table half of the region's rows
+      // (index i at row i/32, column i%32); the table is no longer read
       const int grp = ctid / J;
 #pragma unroll
-      for (int w = 0; w < W; ++w) ored[grp * D + j * W + w] = acc[w];
+      for (int w = 0; w < W; ++w) {
+        const int i = grp * D + j * W + w;
+        lut[(i >> 5) * 64 + (i & 31)] = acc[w];
+      }
       consumer_sync();
       if (ctid < D) {
         float o = 0.f;
 #pragma unroll 8
-        for (int i = 0; i < kGroups; ++i) o += ored[i * D + ctid];
+        for (int i = 0; i < kGroups; ++i) {
+          const int x = i * D + ctid;
+          o += lut[(x >> 5) * 64 + (x & 31)];
+        }
         part[ctid] = o / scaleS;
       }
     }
@@ -665,6 +702,24 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
                    kStageBytes / 4, ctid, kNW * 32);
     if (ctid == 0) atomicExch(p.tickets + unit, 0u);
   }
+}
+
+// Launches the decode kernel as a programmatic dependent of the previous
+// kernel in the stream (it may start while that kernel finishes; the kernel
+// waits for it before touching anything it may write).
+static cudaError_t launch_pdl(const void* fn, dim3 grid, cudaStream_t s, DecodeParams* p) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kDynSmem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  void* args[] = {p};
+  return cudaLaunchKernelExC(&cfg, fn, args);
 }
 
 // Host-side plan: body tokens per split so that the grid fills the SMs.
@@ -779,6 +834,8 @@ extern "C" loopvq_status loopvq_decode_attn(const loopvq_codebook_desc* desc, co
   p.split_len = pl.split_len;
   p.max_splits = pl.max_splits;
 
+  p.static_inputs = (layout->flags & LOOPVQ_LAYOUT_STATIC_INPUTS) ? 1 : 0;
+
   dim3 grid(pl.max_splits, g.Hq, layout->batch);
   cudaStream_t s = (cudaStream_t)stream;
 #define LOOPVQ_LAUNCH(JJ, DD, CBT)                                                                    \
@@ -786,7 +843,7 @@ extern "C" loopvq_status loopvq_decode_attn(const loopvq_codebook_desc* desc, co
     auto kfn = decode_kernel<JJ, DD, CBT>;                                                           \
     if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, kDynSmem) != cudaSuccess) \
       return LOOPVQ_ERR_CUDA;                                                                        \
-    kfn<<<grid, kThreads, kDynSmem, s>>>(p);                                                         \
+    if (launch_pdl((const void*)kfn, grid, s, &p) != cudaSuccess) return LOOPVQ_ERR_CUDA;           \
   } while (0)
 #define LOOPVQ_LAUNCH_J(DD, CBT)                      \
   do {                                                \
@@ -913,13 +970,15 @@ extern "C" loopvq_status loopvq_decode_attn_noalloc(const loopvq_codebook_desc* 
   p.split_len = pl.split_len;
   p.max_splits = pl.max_splits;
 
+  p.static_inputs = (layout->flags & LOOPVQ_LAYOUT_STATIC_INPUTS) ? 1 : 0;
+
   dim3 grid(pl.max_splits, g.Hq, layout->batch);
 #define LOOPVQ_LAUNCH(JJ, DD, CBT)                                                                    \
   do {                                                                                               \
     auto kfn = decode_kernel<JJ, DD, CBT>;                                                           \
     if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, kDynSmem) != cudaSuccess) \
       return LOOPVQ_ERR_CUDA;                                                                        \
-    kfn<<<grid, kThreads, kDynSmem, s>>>(p);                                                         \
+    if (launch_pdl((const void*)kfn, grid, s, &p) != cudaSuccess) return LOOPVQ_ERR_CUDA;           \
   } while (0)
 #define LOOPVQ_LAUNCH_J(DD, CBT)                      \
   do {                                                \

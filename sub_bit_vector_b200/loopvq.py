@@ -32,6 +32,8 @@ LOOPVQ_FAULT_CTX_RANGE = 0x2
 LOOPVQ_FAULT_POOL_RANGE = 0x4
 LOOPVQ_FAULT_TIMEOUT = 0x8
 
+LOOPVQ_LAYOUT_STATIC_INPUTS = 0x1
+
 EXPORTED = [
     "loopvq_version", "loopvq_status_string", "loopvq_validate_desc", "loopvq_ctx_split",
     "loopvq_bits_per_element",
@@ -57,7 +59,7 @@ class loopvq_codebook_desc(ctypes.Structure):
 
 class loopvq_cache_layout(ctypes.Structure):
     _fields_ = [("batch", ctypes.c_int32), ("n_sink", ctypes.c_int32), ("n_recent", ctypes.c_int32),
-                ("page", ctypes.c_int32), ("max_ctx_len", ctypes.c_int32), ("reserved", ctypes.c_int32),
+                ("page", ctypes.c_int32), ("max_ctx_len", ctypes.c_int32), ("flags", ctypes.c_uint32),
                 ("ctx_len", ctypes.c_void_p), ("body_off", ctypes.c_void_p), ("win_off", ctypes.c_void_p),
                 ("body_pool_tokens", ctypes.c_int64), ("win_pool_tokens", ctypes.c_int64)]
 
@@ -148,8 +150,8 @@ def make_desc(n_loop, tc, n_heads_kv, head_dim, group_elems, n_codes=256, n_head
 
 
 def make_layout(batch, n_sink, n_recent, page, max_ctx_len, ctx_len, body_off, win_off,
-                body_pool_tokens, win_pool_tokens) -> loopvq_cache_layout:
-    return loopvq_cache_layout(batch, n_sink, n_recent, page, max_ctx_len, 0, _ptr(ctx_len), _ptr(body_off),
+                body_pool_tokens, win_pool_tokens, flags=0) -> loopvq_cache_layout:
+    return loopvq_cache_layout(batch, n_sink, n_recent, page, max_ctx_len, flags, _ptr(ctx_len), _ptr(body_off),
                                _ptr(win_off), body_pool_tokens, win_pool_tokens)
 
 

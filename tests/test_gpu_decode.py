@@ -33,7 +33,7 @@ class Case:
 
     def __init__(self, *, seed, ctx_lens, H=16, D=128, G=16, Tc=4, T=4, n_sink=64, n_recent=256, page=8,
                  Hq=None, n_codes=256, q_dtype=torch.bfloat16, out_dtype=torch.float32,
-                 cb_dtype=torch.bfloat16, max_ctx_len=None, keep=None):
+                 cb_dtype=torch.bfloat16, max_ctx_len=None, keep=None, static_inputs=False):
         cache, L = _lib()
         self.T, self.Tc, self.H, self.D, self.G = T, Tc, H, D, G
         self.Hq = Hq or H
@@ -45,7 +45,7 @@ class Case:
         self.c = cache.DecodeCache(n_loop=T, tc=Tc, n_heads_kv=H, head_dim=D, group_elems=G, ctx_lens=ctx_lens,
                                    n_sink=n_sink, n_recent=n_recent, page=page, n_codes=n_codes, n_heads_q=self.Hq,
                                    cb_dtype=cb_dtype, q_dtype=q_dtype, out_dtype=out_dtype,
-                                   max_ctx_len=max_ctx_len)
+                                   max_ctx_len=max_ctx_len, static_inputs=static_inputs)
         self.splits = [O.window_split(c, n_sink, n_recent, page) for c in ctx_lens]
         assert [tuple(s) for s in self.splits] == [tuple(s) for s in self.c.splits]
         self.outl = synth.key_outlier_channels(seed, H, D)
@@ -296,6 +296,27 @@ def test_dense_comparator_32k_matches_oracle():
     for h in range(H):
         assert _err(o[h], ref[h]) <= TOL
     np.testing.assert_allclose(ld.cpu().numpy()[0], lref, atol=TOL)
+
+
+def test_static_inputs_flag_back_to_back():
+    """With the static-inputs layout flag the kernel starts streaming codes
+    while the previous launch finishes; back-to-back launches on one stream
+    (all four loop steps, no host sync in between) still match the oracle."""
+    case = Case(seed=26, ctx_lens=[12000, 700, 30000], H=4, static_inputs=True)
+    outs = []
+    for t in range(4):
+        case.c.set_queries(case.q[t])
+        case.c.decode(t)
+        outs.append((case.c.out.clone(), case.c.lse.clone()))
+    torch.cuda.synchronize()
+    for t in range(4):
+        out, lse = outs[t][0].cpu().numpy(), outs[t][1].cpu().numpy()
+        for r in range(3):
+            o_ref, l_ref = case.oracle(t, r)
+            for h in range(4):
+                assert _err(out[r, h], o_ref[h]) <= TOL, (t, r, h)
+                assert abs(lse[r, h] - l_ref[h]) <= TOL * max(1.0, abs(l_ref[h]))
+    assert case.c.device_status()[1] == 0
 
 
 def test_repeated_calls_reuse_workspace():
