@@ -87,15 +87,15 @@ def cpu_baseline(budget_s: float = 15.0):
     tasks of the workload, sized to about `budget_s` seconds of CPU work."""
     import multiprocessing as mp
     cores = _cores()
-    one = _oracle_task((0, 0, 1))
-    n_tasks = max(cores, int(budget_s * cores / max(one, 1e-3)))
-    n_tasks = min(n_tasks, 64 * cores)
-    tasks = [(i % H, (i // H) % T, 1) for i in range(n_tasks)]
     ctx = mp.get_context("spawn")
     with ctx.Pool(cores) as pool:
-        pool.map(_oracle_task, tasks[:cores])      # warm the workers
+        per = pool.map(_oracle_task, [(i % H, 0, 1) for i in range(cores)])   # warm the workers
+        # size the timed sample to ~budget_s of wall time on all cores
+        rounds = max(1, min(16, int(budget_s / max(max(per), 1e-3))))
+        n_tasks = rounds * cores
+        tasks = [(i % H, (i // H) % T, 1) for i in range(n_tasks)]
         t0 = time.perf_counter()
-        pool.map(_oracle_task, tasks)
+        pool.map(_oracle_task, tasks, chunksize=1)
         wall = time.perf_counter() - t0
     return {"value": n_tasks * CTX / wall, "unit": UNIT, "cores": cores, "kind": "oracle",
             "sample": f"{n_tasks} (KV head, loop step) decode-attention problems of the 32K workload "
@@ -226,8 +226,11 @@ def build_layers(device, n_layers):
     W = G // TC
     J = D // W
     for i in range(n_layers):
+        # the layer's pools and codebooks are not written while its decodes run
+        # (the page encode below writes a separate pool), so the kernel may
+        # start streaming them while the previous launch finishes
         c = cache.DecodeCache(n_loop=T, tc=TC, n_heads_kv=H, head_dim=D, group_elems=G, ctx_lens=[CTX],
-                              n_sink=N_SINK, n_recent=N_RECENT, page=PAGE, device=device)
+                              n_sink=N_SINK, n_recent=N_RECENT, page=PAGE, device=device, static_inputs=True)
         outl = synth.key_outlier_channels(100 + i, H, D)
         c.set_codebooks(synth.uniform_codebook(200 + i, T // TC, H, J, 256, TC, W, outlier_channels=outl),
                         synth.uniform_codebook(300 + i, T // TC, H, J, 256, TC, W))
@@ -287,6 +290,24 @@ def dense_comparator(device, reps=50):
     by = 2 * H * CTX * D * 2 + H * D * 2 + H * D * 4
     return {"us_per_launch": us, "bytes_per_launch": by, "GB_per_s": by / us / 1e3,
             "kv_tokens_per_s": CTX / (us * 1e-6)}
+
+
+def reduce_over_ranks(values, world, device=None):
+    """Max over ranks of per-rank device timings (ms); every rank takes the
+    same collective step.  Returns the list of maxima."""
+    if world <= 1:
+        return list(values)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
+def aggregate_value(world, steps, tokens_per_step, elapsed_ms):
+    """Whole-job throughput: every rank processed `steps` steps of its own
+    workload (weak scaling) within the max-over-ranks time."""
+    return world * steps * tokens_per_step / (elapsed_ms * 1e-3)
 
 
 def run_gpu(args):
@@ -364,14 +385,11 @@ def run_gpu(args):
     elapsed_ms = start.elapsed_time(end)
     decode_ms = sum(a.elapsed_time(b) for a, b in evs)
     n_enc_steps = sum(1 for i in range(args.steps) if i % PAGE == PAGE - 1)
-    if world > 1:
-        t = torch.tensor([elapsed_ms, decode_ms], dtype=torch.float64, device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms, decode_ms = float(t[0]), float(t[1])
+    elapsed_ms, decode_ms = reduce_over_ranks([elapsed_ms, decode_ms], world, device)
 
     status = [c.device_status()[1] for c in layers]
     tokens_per_step = CTX * T
-    value = world * args.steps * tokens_per_step / (elapsed_ms * 1e-3)
+    value = aggregate_value(world, args.steps, tokens_per_step, elapsed_ms)
     algo = layers[0].algorithmic_bytes()
     us_launch = decode_ms * 1e3 / (args.steps * T)
     peak, peak_kind = _peak_hbm()
@@ -420,12 +438,8 @@ def run_gpu(args):
             e2e_step(i)
         s1.record(stream)
         torch.cuda.synchronize()
-    e2e_ms = s0.elapsed_time(s1)
-    if world > 1:
-        t = torch.tensor([e2e_ms], dtype=torch.float64, device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t[0])
-    e2e = {"value": world * e2e_steps * tokens_per_step / (e2e_ms * 1e-3), "unit": UNIT,
+    e2e_ms = reduce_over_ranks([s0.elapsed_time(s1)], world, device)[0]
+    e2e = {"value": aggregate_value(world, e2e_steps, tokens_per_step, e2e_ms), "unit": UNIT,
            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": e2e_steps,
            "path": "pinned host q + new-token K/V -> device, 4 loopvq_decode_attn calls (+ page encode every "
                    "8th step), fp32 outputs -> pinned host, stream sync per step"}

@@ -30,6 +30,8 @@
 #include <math.h>
 #include <stdio.h>
 
+#include <utility>
+
 #include "common.cuh"
 
 namespace loopvq {
@@ -39,13 +41,15 @@ constexpr int kThreads = (kNW + 1) * 32;     // + one producer warp
 constexpr int kStages = 4;
 constexpr int kStageBytes = 32768;
 constexpr int kSplitCap = 4064;              // max body tokens per split, multiple of 32
-// The lookup table and the histogram share one 64 KB region of 256 rows (one
-// per code) of 256 bytes: 32 fp32 table columns, then 32 u32 histogram
-// columns.  The region is 64 KB aligned in the shared window, so the shared
-// address of (code, column) is a single byte permute: code in byte 1, the
-// column offset in byte 0, the region base in bytes 2-3.
+// One 64 KB region of 256 rows (one per code) of 64 four-byte columns holds
+// the lookup table during pass K and the histogram during pass V.  Column x
+// stands for slot x mod J (the table is replicated 64/J times), so lane l at
+// step s uses column l + s: 32 distinct banks, no wrap-around.  The region is
+// 64 KB aligned in the shared window, so the address of (code, column l) is a
+// single byte permute (code in byte 1, l*4 in byte 0, the region base in
+// bytes 2-3) and the step's 4*s is the load's immediate offset.
 constexpr int kRegionBytes = 65536;
-constexpr int kHistColOff = 128;             // histogram column offset in a row
+constexpr int kCols = 64;
 constexpr int kScoresBytes = kSplitCap * 4;
 constexpr int kMiscBytes = 4096;
 // allocation: the region, the ring, scores and misc, plus room to align the
@@ -101,10 +105,15 @@ __device__ __forceinline__ float lds_f32(uint32_t a) {
   asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(a));
   return v;
 }
-// the histogram bin sits kHistColOff bytes after the table entry of the same
-// code and column
-__device__ __forceinline__ void red_hist_u32(uint32_t lut_addr, uint32_t v) {
-  asm volatile("red.shared.add.u32 [%0+128], %1;" ::"r"(lut_addr), "r"(v) : "memory");
+template <int OFF>
+__device__ __forceinline__ float lds_f32_off(uint32_t a) {
+  float v;
+  asm volatile("ld.shared.f32 %0, [%1+%2];" : "=f"(v) : "r"(a), "n"(OFF));
+  return v;
+}
+template <int OFF>
+__device__ __forceinline__ void red_u32_off(uint32_t a, uint32_t v) {
+  asm volatile("red.shared.add.u32 [%0+%1], %2;" ::"r"(a), "n"(OFF), "r"(v) : "memory");
 }
 // acc (two packed fp32) += (x, y)
 __device__ __forceinline__ uint64_t add_f32x2(uint64_t acc, float x, float y) {
@@ -136,62 +145,79 @@ __device__ __forceinline__ void load_tile_words(const uint8_t* tile, int lane, u
   }
 }
 
-// Shared address of the lookup-table entry of code = byte K of w for the
-// lane's column at that step: col holds the region base (bytes 2-3) and the
-// column offset (byte 0); the code becomes byte 1 (row of 256 bytes).
+// Shared address of (code = byte K of w, column lane): lb holds the region
+// base (bytes 2-3) and lane*4 (byte 0); the code becomes byte 1.
 template <int K>
-__device__ __forceinline__ uint32_t entry_addr(uint32_t w, uint32_t col) {
-  return __byte_perm(w, col, 0x7604u | (K << 4));
+__device__ __forceinline__ uint32_t code_addr(uint32_t w, uint32_t lb) {
+  return __byte_perm(w, lb, 0x7604u | (K << 4));
+}
+
+// Word I of a lane's codes (steps 4I .. 4I+3) for two tiles: gathers of
+// table columns lane + s (immediate offset 4s) into packed fp32 pair sums.
+template <int I>
+__device__ __forceinline__ void score_word(uint32_t w0, uint32_t w1, uint32_t lb, uint64_t& a01, uint64_t& a23,
+                                           uint64_t& b01, uint64_t& b23) {
+  const float x0 = lds_f32_off<16 * I + 0>(code_addr<0>(w0, lb));
+  const float y0 = lds_f32_off<16 * I + 0>(code_addr<0>(w1, lb));
+  const float x1 = lds_f32_off<16 * I + 4>(code_addr<1>(w0, lb));
+  const float y1 = lds_f32_off<16 * I + 4>(code_addr<1>(w1, lb));
+  const float x2 = lds_f32_off<16 * I + 8>(code_addr<2>(w0, lb));
+  const float y2 = lds_f32_off<16 * I + 8>(code_addr<2>(w1, lb));
+  const float x3 = lds_f32_off<16 * I + 12>(code_addr<3>(w0, lb));
+  const float y3 = lds_f32_off<16 * I + 12>(code_addr<3>(w1, lb));
+  a01 = add_f32x2(a01, x0, x1);
+  b01 = add_f32x2(b01, y0, y1);
+  a23 = add_f32x2(a23, x2, x3);
+  b23 = add_f32x2(b23, y2, y3);
+}
+template <int N, int... Is>
+__device__ __forceinline__ void score_words(const uint32_t (&w0)[N], const uint32_t (&w1)[N], uint32_t lb,
+                                            uint64_t& a01, uint64_t& a23, uint64_t& b01, uint64_t& b23,
+                                            std::integer_sequence<int, Is...>) {
+  (score_word<Is>(w0[Is], w1[Is], lb, a01, a23, b01, b23), ...);
 }
 
 // Scores of this lane's token in two tiles at once (two independent chains
-// for latency hiding): the sum over its J codes of the lookup-table column
-// the rotation assigns to each step.
+// for latency hiding): the sum over its J codes of table column lane + s at
+// step s, i.e. slot (s + lane) mod J, which is the tile's byte order.
 template <int J>
-__device__ __forceinline__ void token_score2(const uint8_t* t0, const uint8_t* t1, int lane,
-                                             const uint32_t (&col)[J], float& s0, float& s1) {
+__device__ __forceinline__ void token_score2(const uint8_t* t0, const uint8_t* t1, int lane, uint32_t lb,
+                                             float& s0, float& s1) {
   uint32_t w0[J / 4], w1[J / 4];
   load_tile_words<J>(t0, lane, w0);
   load_tile_words<J>(t1, lane, w1);
   uint64_t a01 = 0, a23 = 0, b01 = 0, b23 = 0;   // packed fp32 pairs, 0 bits = (0, 0)
-#pragma unroll
-  for (int i = 0; i < J / 4; ++i) {
-    const float x0 = lds_f32(entry_addr<0>(w0[i], col[4 * i + 0]));
-    const float y0 = lds_f32(entry_addr<0>(w1[i], col[4 * i + 0]));
-    const float x1 = lds_f32(entry_addr<1>(w0[i], col[4 * i + 1]));
-    const float y1 = lds_f32(entry_addr<1>(w1[i], col[4 * i + 1]));
-    const float x2 = lds_f32(entry_addr<2>(w0[i], col[4 * i + 2]));
-    const float y2 = lds_f32(entry_addr<2>(w1[i], col[4 * i + 2]));
-    const float x3 = lds_f32(entry_addr<3>(w0[i], col[4 * i + 3]));
-    const float y3 = lds_f32(entry_addr<3>(w1[i], col[4 * i + 3]));
-    a01 = add_f32x2(a01, x0, x1);
-    b01 = add_f32x2(b01, y0, y1);
-    a23 = add_f32x2(a23, x2, x3);
-    b23 = add_f32x2(b23, y2, y3);
-  }
+  score_words(w0, w1, lb, a01, a23, b01, b23, std::make_integer_sequence<int, J / 4>{});
   s0 = sum_f32x2(a01) + sum_f32x2(a23);
   s1 = sum_f32x2(b01) + sum_f32x2(b23);
 }
 
+template <int I>
+__device__ __forceinline__ void hist_word(uint32_t w0, uint32_t w1, uint32_t lb, uint32_t q0, uint32_t q1) {
+  red_u32_off<16 * I + 0>(code_addr<0>(w0, lb), q0);
+  red_u32_off<16 * I + 0>(code_addr<0>(w1, lb), q1);
+  red_u32_off<16 * I + 4>(code_addr<1>(w0, lb), q0);
+  red_u32_off<16 * I + 4>(code_addr<1>(w1, lb), q1);
+  red_u32_off<16 * I + 8>(code_addr<2>(w0, lb), q0);
+  red_u32_off<16 * I + 8>(code_addr<2>(w1, lb), q1);
+  red_u32_off<16 * I + 12>(code_addr<3>(w0, lb), q0);
+  red_u32_off<16 * I + 12>(code_addr<3>(w1, lb), q1);
+}
+template <int N, int... Is>
+__device__ __forceinline__ void hist_words(const uint32_t (&w0)[N], const uint32_t (&w1)[N], uint32_t lb, uint32_t q0,
+                                           uint32_t q1, std::integer_sequence<int, Is...>) {
+  (hist_word<Is>(w0[Is], w1[Is], lb, q0, q1), ...);
+}
+
 // Adds this lane's token weights of two tiles into the histogram bins of
-// their codes.
+// their codes (same columns as the scores).
 template <int J>
-__device__ __forceinline__ void token_hist2(const uint8_t* t0, const uint8_t* t1, int lane,
-                                            const uint32_t (&col)[J], uint32_t q0, uint32_t q1) {
+__device__ __forceinline__ void token_hist2(const uint8_t* t0, const uint8_t* t1, int lane, uint32_t lb,
+                                            uint32_t q0, uint32_t q1) {
   uint32_t w0[J / 4], w1[J / 4];
   load_tile_words<J>(t0, lane, w0);
   load_tile_words<J>(t1, lane, w1);
-#pragma unroll
-  for (int i = 0; i < J / 4; ++i) {
-    red_hist_u32(entry_addr<0>(w0[i], col[4 * i + 0]), q0);
-    red_hist_u32(entry_addr<0>(w1[i], col[4 * i + 0]), q1);
-    red_hist_u32(entry_addr<1>(w0[i], col[4 * i + 1]), q0);
-    red_hist_u32(entry_addr<1>(w1[i], col[4 * i + 1]), q1);
-    red_hist_u32(entry_addr<2>(w0[i], col[4 * i + 2]), q0);
-    red_hist_u32(entry_addr<2>(w1[i], col[4 * i + 2]), q1);
-    red_hist_u32(entry_addr<3>(w0[i], col[4 * i + 3]), q0);
-    red_hist_u32(entry_addr<3>(w1[i], col[4 * i + 3]), q1);
-  }
+  hist_words(w0, w1, lb, q0, q1, std::make_integer_sequence<int, J / 4>{});
 }
 
 // Loads W consecutive codebook elements (bf16 or fp32) as fp32; zero if !ok.
@@ -342,8 +368,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
     return;
   }
   uint8_t* const region_p = dyn + (region - sbase);
-  float* const lut = reinterpret_cast<float*>(region_p);         // row c: lut[c*64 + col]
-  uint32_t* const hist = reinterpret_cast<uint32_t*>(region_p);  // row c: hist[c*64 + 32 + col]
+  float* const lut = reinterpret_cast<float*>(region_p);         // pass K: lut[c*64 + col]
+  uint32_t* const hist = reinterpret_cast<uint32_t*>(region_p);  // pass V: hist[c*64 + col]
   auto stage_ptr = [&](int i) -> uint8_t* { return dyn + (stage_a[i] - sbase); };
   float* const sc = reinterpret_cast<float*>(dyn + (sc_a - sbase));
   uint8_t* const misc = dyn + (misc_a - sbase);
@@ -530,14 +556,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
         for (int w = 0; w < W; ++w) acc = fmaf(qj[w], wk[k][w], acc);
         if (c >= p.C) acc = __int_as_float(0x7fc00000);  // NaN marks a code >= n_codes
 #pragma unroll
-        for (int g = 0; g < 32 / J; ++g) lut[c * 64 + g * J + j] = acc;
+        for (int g = 0; g < kCols / J; ++g) lut[c * kCols + g * J + j] = acc;
       }
     }
-    for (int e = ctid; e < 256 * 32; e += kNW * 32) hist[(e >> 5) * 64 + 32 + (e & 31)] = 0u;
-    // this lane's column at step s: (lane / J) * J + (s + lane) mod J
-    uint32_t col[J];
-#pragma unroll
-    for (int s = 0; s < J; ++s) col[s] = region | (uint32_t)(((lane / J) * J + ((s + lane) % J)) * 4);
+    const uint32_t lb = region | (uint32_t)(lane * 4);
     consumer_sync();
 
     // ---- pass K: scores and split maximum
@@ -551,7 +573,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
       for (int tl = warp; tl < nt; tl += 2 * kNW) {
         const int tl2 = tl + kNW < nt ? tl + kNW : tl;
         float sv0, sv1;
-        token_score2<J>(st + tl * 32 * J, st + tl2 * 32 * J, lane, col, sv0, sv1);
+        token_score2<J>(st + tl * 32 * J, st + tl2 * 32 * J, lane, lb, sv0, sv1);
         const int tok0c = (k * kTilesPerChunk + tl) * 32 + lane;
         const bool v0 = tok0c < n_tok;
         if (v0 && sv0 != sv0) nan_seen = true;
@@ -575,6 +597,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
     consumer_sync();
     float m = -INFINITY;
     for (int w = 0; w < kNW; ++w) m = fmaxf(m, red[w]);
+    // the table is done with: the region becomes the histogram
+    for (int e = ctid; e < 256 * kCols / 4; e += kNW * 32) reinterpret_cast<uint4*>(hist)[e] = make_uint4(0u, 0u, 0u, 0u);
+    consumer_sync();
     // fixed-point scale: n_tok * 2^S < 2^32 with S = clz(n_tok)
     const int S = __clz(max(n_tok, 1));
     const float scaleS = exp2f((float)S);
@@ -602,7 +627,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
           }
           qsum += qv[u];
         }
-        token_hist2<J>(st + tl * 32 * J, st + tl2 * 32 * J, lane, col, qv[0], qv[1]);
+        token_hist2<J>(st + tl * 32 * J, st + tl2 * 32 * J, lane, lb, qv[0], qv[1]);
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(empty_bar + s));
@@ -634,7 +659,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
     // 512/J partial groups per output are summed through shared memory (the
     // LUT region is free by now).
     {
-      constexpr int kGroups = (kNW * 32) / J;
       float acc[W];
 #pragma unroll
       for (int w = 0; w < W; ++w) acc[w] = 0.f;
@@ -644,7 +668,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
         const int c = (ctid + k * kNW * 32) / J;
         uint32_t hs = 0;
 #pragma unroll
-        for (int g = 0; g < 32 / J; ++g) hs += hist[c * 64 + 32 + g * J + j];
+        for (int g = 0; g < kCols / J; ++g) hs += hist[c * kCols + g * J + j];
         if (c < p.C && hs != 0u) {
           const float hf = (float)hs;
 #pragma unroll
@@ -654,25 +678,25 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
       // bins of codes >= n_codes must be empty
       if (p.C < 256) {
         bool any = false;
-        for (int e = p.C * 32 + ctid; e < 256 * 32; e += kNW * 32) any |= hist[(e >> 5) * 64 + 32 + (e & 31)] != 0u;
+        for (int e = p.C * kCols + ctid; e < 256 * kCols; e += kNW * 32) any |= hist[e] != 0u;
         if (any) set_fault(p.status, LOOPVQ_FAULT_CODE_RANGE);
       }
-      // [kGroups][D] partial sums in the table half of the region's rows
-      // (index i at row i/32, column i%32); the table is no longer read
-      const int grp = ctid / J;
+      // lanes l and l + J of a warp hold the same slot: fold them first
 #pragma unroll
-      for (int w = 0; w < W; ++w) {
-        const int i = grp * D + j * W + w;
-        lut[(i >> 5) * 64 + (i & 31)] = acc[w];
+      for (int o = J; o < 32; o <<= 1) {
+#pragma unroll
+        for (int w = 0; w < W; ++w) acc[w] += __shfl_xor_sync(0xffffffffu, acc[w], o);
+      }
+      float* ored = sc;  // [kNW][D] per-warp partial sums; scores are no longer read
+      if (lane < J) {
+#pragma unroll
+        for (int w = 0; w < W; ++w) ored[warp * D + j * W + w] = acc[w];
       }
       consumer_sync();
       if (ctid < D) {
         float o = 0.f;
-#pragma unroll 8
-        for (int i = 0; i < kGroups; ++i) {
-          const int x = i * D + ctid;
-          o += lut[(x >> 5) * 64 + (x & 31)];
-        }
+#pragma unroll
+        for (int i = 0; i < kNW; ++i) o += ored[i * D + ctid];
         part[ctid] = o / scaleS;
       }
     }
