@@ -30,6 +30,7 @@ import argparse
 import hashlib
 import json
 import os
+import re
 import subprocess
 import sys
 import time
@@ -202,13 +203,17 @@ def _decode_src_hash():
 
 def _profiled_traffic():
     """DRAM bytes per decode launch from the committed ncu summary, if it was
-    taken on the current kernel source."""
-    p = os.path.join(ROOT, "profiles", "decode_kernel_ouro14_32k_half_bit.json")
+    taken on the current kernel source (the summary names the source hash)."""
+    p = os.path.join(ROOT, "profiles", "decode_kernel_ouro14_32k_half_bit.md")
     try:
-        d = json.load(open(p))
-    except Exception:
+        text = open(p).read()
+    except OSError:
         return None
-    return d.get("traffic_bytes_per_launch") if d.get("decode_src_sha256_16") == _decode_src_hash() else None
+    m_t = re.search(r"traffic_bytes_per_launch:\s*(\d+)", text)
+    m_h = re.search(r"decode_src_sha256_16:\s*([0-9a-f]{16})", text)
+    if not m_t or not m_h or m_h.group(1) != _decode_src_hash():
+        return None
+    return int(m_t.group(1))
 
 
 def _peak_hbm():

@@ -209,8 +209,7 @@ LOOPVQ_API loopvq_status loopvq_index_pool_unpack(const loopvq_codebook_desc* de
  * KV head h, slot j and token n, forms the sub-vector
  *   x[tt*W + w] = X[b*Tc + tt][n][h][j*W + w],  tt < Tc, w < W
  * and stores argmin_c sum_g (x[g] - codeword_c[g])^2 over c < n_codes, ties
- * to the lowest c (distances in fp32 from the differences), at pool position
- * tok_off + n.
+ * to the lowest c, at pool position tok_off + n.
  *   cb_packed : device, from loopvq_codebook_pack (this stream's kind).
  *   x         : device, element (t, n, h, d) at
  *               x[t*stride_t + n*stride_n + h*stride_h + d] in x_dtype; d is
@@ -220,12 +219,26 @@ LOOPVQ_API loopvq_status loopvq_index_pool_unpack(const loopvq_codebook_desc* de
  *   kind      : the stream written (K and V tiles differ in byte order).
  *   idx_pool  : device, loopvq_index_pool_bytes(desc, pool_tokens) bytes.
  * n_tokens = 0 is a no-op.  tok_off + n_tokens must not exceed pool_tokens.
+ * Kernels: bf16 x with a bf16 256-entry codebook, G in {16, 32}, W a multiple
+ * of 4, x 8-byte aligned, strides multiples of 4 and n_tokens >= 256 run on
+ * the tensor cores (tcgen05: d = |x|^2 + |c|^2 - 2 x.c in fp32, with every
+ * near-tie re-solved exactly from the differences); everything else runs the
+ * CUDA-core kernel.  Both return the nearest codeword up to fp32 rounding of
+ * distances that are equal within it.  A device-side timeout (never expected)
+ * leaves that tile's codes unwritten and sets LOOPVQ_FAULT_TIMEOUT in the
+ * word read by loopvq_read_encode_faults.
  */
 LOOPVQ_API loopvq_status loopvq_encode(const loopvq_codebook_desc* desc, const void* cb_packed,
                             loopvq_kind kind, const void* x, loopvq_dtype x_dtype,
                             int64_t n_tokens, int64_t stride_t, int64_t stride_n,
                             int64_t stride_h, uint8_t* idx_pool, int64_t tok_off,
                             int64_t pool_tokens, loopvq_stream_t stream);
+
+/* Waits for `stream`, then reads the encoder's device fault word (one per
+ * device, shared by all encode calls): LOOPVQ_OK if zero, else
+ * LOOPVQ_ERR_DEVICE_FAULT with the LOOPVQ_FAULT_* bits in *bits (if non-NULL).
+ * clear != 0 zeroes the word afterwards. */
+LOOPVQ_API loopvq_status loopvq_read_encode_faults(uint32_t* bits, int32_t clear, loopvq_stream_t stream);
 
 /* ---------------------------------------------------------------- decode */
 

@@ -1,0 +1,412 @@
+// Loop-axis VQ encode on the 5th-generation tensor cores (sm_100a).
+//
+// LoopVQ project page, "Method" -- "Overview of LoopVQ" and "Component 1":
+// each loop-axis sub-vector x (G elements: W channels of each of Tc
+// consecutive loop steps) is replaced by the index of its nearest codeword.
+// For bf16 inputs and 256-entry bf16 codebooks the distance block is a dense
+// contraction,
+//
+//   d(n, c) = ||x_n||^2 + ||c||^2 - 2 x_n . c ,
+//
+// computed for a tile of 128 sub-vectors x 256 codewords by tcgen05.mma (bf16
+// operands in shared memory, fp32 accumulator in tensor memory).  The norms
+// ride in the contraction: K is padded from G to a multiple of 16 and the pad
+// holds each norm split exactly into three bf16 parts (hi + mid + lo equals
+// the fp32 value) against ones on the other operand, so the accumulator holds
+// d itself.  Every product of two bf16 values is exact in fp32; only the sums
+// round.
+//
+// Epilogue (one thread per sub-vector = one TMEM lane): the row's norm
+// carries a small positive bias (the same for every codeword) that keeps the
+// fast distances positive, so the key "float bits of d with the low 8 bits
+// replaced by the code" orders like d as a signed integer and breaks ties by
+// code; each thread keeps the two smallest keys.  When the two
+// are closer than twice a bound on the fast path's error (plus the 8
+// truncated mantissa bits), the warp re-reads the row from TMEM and the
+// thread re-solves exactly, in fp32 from the differences sum_g (x_g - c_g)^2
+// with a strict "<" in code order, over every codeword whose fast distance is
+// within that bound of the minimum.  The result is the nearest codeword
+// except where two are within fp32 rounding of each other -- the guarantee of
+// the CUDA-core encoder.
+
+#include "common.cuh"
+
+namespace loopvq {
+
+constexpr int kTcTile = 128;        // sub-vectors per MMA tile (M)
+constexpr int kTcCodes = 256;       // codewords (N)
+constexpr int kTcThreads = 128;     // one thread per tile row
+constexpr int kTcTilesPerCta = 32;  // 4096 tokens per CTA
+// Shared memory asked per CTA: at most two CTAs share an SM, so their two
+// 256-column accumulators fit the SM's 512 TMEM columns and tcgen05.alloc
+// never has to wait for another CTA.
+constexpr int kTcSmemFloor = 80 * 1024;
+
+struct EncodeTcParams {
+  const __nv_bfloat16* x;
+  int64_t st, sn, sh;  // element strides of t, n, h
+  int64_t n_tokens;
+  const __nv_bfloat16* cb;  // canonical [NB][H][J][C][Tc][W]
+  int Tc, H, J, W, kind;
+  uint8_t* pool;
+  int64_t tok_off, pool_tokens;
+};
+
+__device__ uint32_t g_encode_faults;
+
+// ---- canonical K-major, no-swizzle operand layout ---------------------------
+// A [rows][KP] bf16 operand is stored as 8-row x 16-byte core matrices of 128
+// contiguous bytes; core (r/8, k/8) sits at (r/8)*SBO + (k/8)*LBO with
+// LBO = 128 B (next 8 elements of K) and SBO = KP/8 * 128 B (next 8 rows).
+template <int KP>
+__device__ __forceinline__ uint32_t core_off(int r, int k8) {
+  return (uint32_t)((r >> 3) * (KP / 8) * 128 + k8 * 128 + (r & 7) * 16);
+}
+template <int KP>
+__device__ __forceinline__ uint64_t umma_smem_desc(uint32_t saddr) {
+  constexpr uint64_t lbo = 128, sbo = (KP / 8) * 128;
+  uint64_t d = (uint64_t)((saddr >> 4) & 0x3FFF);
+  d |= ((lbo >> 4) & 0x3FFF) << 16;
+  d |= ((sbo >> 4) & 0x3FFF) << 32;
+  d |= (uint64_t)1 << 46;  // sm_100 descriptor version; base offset 0, no swizzle
+  return d;
+}
+// kind::f16 instruction descriptor: fp32 accumulator, bf16 A and B, both
+// K-major, N = 256, M = 128.
+constexpr uint32_t kTcIdesc =
+    (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kTcCodes >> 3) << 17) | ((uint32_t)(kTcTile >> 4) << 24);
+
+__device__ __forceinline__ void umma_f16(uint32_t dtmem, uint64_t ad, uint64_t bd, uint32_t acc) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(dtmem),
+      "l"(ad), "l"(bd), "r"(kTcIdesc), "r"(acc)
+      : "memory");
+}
+__device__ __forceinline__ void umma_commit(uint32_t mbar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(mbar) : "memory");
+}
+__device__ __forceinline__ void tmem_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tmem_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]),
+        "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr)
+      : "memory");
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&v);
+}
+// Exact three-part bf16 split of an fp32 value v >= 0: v == hi + mid + lo.
+__device__ __forceinline__ void split3(float v, float& hi, float& mid, float& lo) {
+  hi = __bfloat162float(__float2bfloat16_rn(v));
+  const float r1 = v - hi;
+  mid = __bfloat162float(__float2bfloat16_rn(r1));
+  lo = __bfloat162float(__float2bfloat16_rn(r1 - mid));
+}
+// Pad words of a row: 16-byte chunks k8 = G/8 .. KP/8-1 (6 used elements).
+// A rows hold [xx_hi xx_mid xx_lo 1 1 1 0 ...], B rows [1 1 1 nc_hi nc_mid nc_lo 0 ...].
+template <int KP, int G>
+__device__ __forceinline__ void write_pad(uint8_t* base, int r, float a0, float a1, float a2, float b0, float b1,
+                                          float b2) {
+  const uint4 w0 = make_uint4(pack_bf16(a0, a1), pack_bf16(a2, b0), pack_bf16(b1, b2), 0u);
+  *reinterpret_cast<uint4*>(base + core_off<KP>(r, G / 8)) = w0;
+#pragma unroll
+  for (int k8 = G / 8 + 1; k8 < KP / 8; ++k8) *reinterpret_cast<uint4*>(base + core_off<KP>(r, k8)) = make_uint4(0u, 0u, 0u, 0u);
+}
+
+template <int G, int KP>
+__global__ void __launch_bounds__(kTcThreads, 2) encode_tc_kernel(const EncodeTcParams p) {
+  extern __shared__ __align__(1024) uint8_t dyn[];
+  constexpr uint32_t kBBytes = kTcCodes * KP * 2;
+  constexpr uint32_t kABytes = kTcTile * KP * 2;
+  uint8_t* const bsm = dyn;
+  uint8_t* const asmem = dyn + kBBytes;
+  uint64_t* const mbar = reinterpret_cast<uint64_t*>(dyn + kBBytes + kABytes);
+  uint32_t* const tmem_slot = reinterpret_cast<uint32_t*>(mbar + 1);
+  int* const nc_max_bits = reinterpret_cast<int*>(tmem_slot + 1);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int j = blockIdx.x;
+  const int bh = blockIdx.z;
+  const int b = bh / p.H, h = bh % p.H;
+  const int64_t tile0 = (int64_t)blockIdx.y * kTcTilesPerCta;
+  const int64_t n_tiles_total = (p.n_tokens + kTcTile - 1) / kTcTile;
+  const int64_t left = n_tiles_total - tile0;
+  const int n_tiles = left < kTcTilesPerCta ? (int)left : kTcTilesPerCta;
+  if (n_tiles <= 0) return;  // uniform across the CTA, before any allocation
+
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"(kTcCodes));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  if (tid == 0) {
+    mbar_init(smem_u32(mbar), 1);
+    *nc_max_bits = 0;
+    fence_mbar_init();
+  }
+
+  // ---- B operand: row c = [-2c (G) | 1 1 1 nc_hi nc_mid nc_lo | 0 ...] ----
+  const __nv_bfloat16* cbp = p.cb + (((int64_t)bh * p.J + j) * kTcCodes) * G;
+  float ncmax = 0.f;
+#pragma unroll 1
+  for (int c = tid; c < kTcCodes; c += kTcThreads) {
+    const uint4* src = reinterpret_cast<const uint4*>(cbp + (int64_t)c * G);
+    float nc = 0.f;
+#pragma unroll
+    for (int k8 = 0; k8 < G / 8; ++k8) {
+      const uint4 v = __ldg(src + k8);
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+      uint32_t o[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float lo = bf16_lo(w[i]), hi = bf16_hi(w[i]);
+        nc = fmaf(lo, lo, nc);
+        nc = fmaf(hi, hi, nc);
+        o[i] = pack_bf16(-2.f * lo, -2.f * hi);  // exact: a power-of-two scale of a bf16 value
+      }
+      *reinterpret_cast<uint4*>(bsm + core_off<KP>(c, k8)) = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+    float hi, mid, lo;
+    split3(nc, hi, mid, lo);
+    write_pad<KP, G>(bsm, c, 1.f, 1.f, 1.f, hi, mid, lo);
+    ncmax = fmaxf(ncmax, nc);
+  }
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) ncmax = fmaxf(ncmax, __shfl_xor_sync(0xffffffffu, ncmax, o));
+  __syncthreads();  // nc_max_bits initialised
+  if (lane == 0) atomicMax(nc_max_bits, __float_as_int(ncmax));  // non-negative floats order as ints
+  tmem_fence_before();
+  __syncthreads();
+  tmem_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const float nc_max = __int_as_float(*nc_max_bits);
+  const uint32_t a_addr = smem_u32(asmem), b_addr = smem_u32(bsm);
+  const uint32_t t_row = tmem + ((uint32_t)(warp * 32) << 16);  // this warp's 32 TMEM lanes
+
+  // ---- sub-vector loads: G/4 groups of 4 consecutive channels (W % 4 == 0) ----
+  const int row = tid;
+  uint2 xr[G / 4];
+  int64_t n_next = tile0 * kTcTile + row;
+  auto load_x = [&](int64_t n) {
+#pragma unroll
+    for (int q = 0; q < G / 4; ++q) {
+      const int g = q * 4, t = g / p.W, w = g - t * p.W;
+      xr[q] = make_uint2(0u, 0u);
+      if (n < p.n_tokens)
+        xr[q] = __ldg(reinterpret_cast<const uint2*>(p.x + (int64_t)(b * p.Tc + t) * p.st + n * p.sn +
+                                                     (int64_t)h * p.sh + (int64_t)j * p.W + w));
+    }
+  };
+  load_x(n_next);
+
+  uint32_t phase = 0;
+#pragma unroll 1
+  for (int tile = 0; tile < n_tiles; ++tile) {
+    const int64_t n = n_next;
+    const bool ok = n < p.n_tokens;
+    // A row: the sub-vector's bf16 words as loaded, then the norm parts
+    float xx = 0.f;
+#pragma unroll
+    for (int k8 = 0; k8 < G / 8; ++k8) {
+      const uint2 u0 = xr[2 * k8], u1 = xr[2 * k8 + 1];
+      *reinterpret_cast<uint4*>(asmem + core_off<KP>(row, k8)) = make_uint4(u0.x, u0.y, u1.x, u1.y);
+      const uint32_t w[4] = {u0.x, u0.y, u1.x, u1.y};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        xx = fmaf(bf16_lo(w[i]), bf16_lo(w[i]), xx);
+        xx = fmaf(bf16_hi(w[i]), bf16_hi(w[i]), xx);
+      }
+    }
+    // Fast-path error bound: the fp32 norms and the tensor core's fp32 sums,
+    // each within a few units of 2^-24 of the sum of the terms' magnitudes
+    // (at most 2 (||x||^2 + ||c||^2)); taken as 2^-15 (||x||^2 + max ||c||^2).
+    const float err = 3.0517578e-5f * (xx + nc_max);
+    {
+      // the row's norm carries a bias of 2 err, equal for every codeword, so
+      // the fast distances stay positive and order as signed integers
+      float hi, mid, lo;
+      split3(xx + 2.f * err, hi, mid, lo);
+      write_pad<KP, G>(asmem, row, hi, mid, lo, 1.f, 1.f, 1.f);
+    }
+    // generic-proxy writes of A (and, the first time, B) -> tensor core
+    fence_proxy_async();
+    tmem_fence_before();
+    __syncthreads();
+    tmem_fence_after();
+    if (tid == 0) {
+#pragma unroll
+      for (int k = 0; k < KP / 16; ++k)
+        umma_f16(tmem, umma_smem_desc<KP>(a_addr + k * 256), umma_smem_desc<KP>(b_addr + k * 256), k > 0 ? 1u : 0u);
+      umma_commit(smem_u32(mbar));
+    }
+    // next tile's loads fly while the MMA runs
+    n_next += kTcTile;
+    if (tile + 1 < n_tiles) load_x(n_next);
+
+    const bool done = mbar_wait_bounded(smem_u32(mbar), phase);
+    if (__syncthreads_or(!done)) {
+      // never expected: record it, give the MMA one more bounded wait so no
+      // tensor-core write is in flight, then leave (codes of this tile unwritten)
+      if (tid == 0) atomicOr(&g_encode_faults, LOOPVQ_FAULT_TIMEOUT);
+      mbar_wait_bounded(smem_u32(mbar), phase);
+      break;
+    }
+    phase ^= 1u;
+    tmem_fence_after();
+
+    // top-2 keys: within a 32-column chunk the key carries the column in its
+    // low 5 bits (an immediate); the chunk number joins in bits 5..7 when a
+    // chunk's top-2 merges into the row's
+    int k1 = 0x7FFFFFFF, k2 = 0x7FFFFFFF;
+#pragma unroll 1
+    for (int cc = 0; cc < kTcCodes / 32; cc += 2) {
+      uint32_t r[2][32];
+      tmem_ld32(t_row + (uint32_t)(cc * 32), r[0]);
+      tmem_ld32(t_row + (uint32_t)(cc * 32 + 32), r[1]);
+      tmem_wait_ld();
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        // two chains of candidate pairs; a pair (lo <= hi) merges into a
+        // chain's sorted (x1 <= x2) as x2 = min(max(x1, lo), x2, hi), x1 = min(x1, lo)
+        int a1 = 0x7FFFFFFF, a2 = 0x7FFFFFFF, b1 = 0x7FFFFFFF, b2 = 0x7FFFFFFF;
+#pragma unroll
+        for (int q = 0; q < 32; q += 4) {
+          const int ka0 = (int)((r[u][q] & 0xFFFFFF00u) | (uint32_t)q);
+          const int ka1 = (int)((r[u][q + 1] & 0xFFFFFF00u) | (uint32_t)(q + 1));
+          const int kb0 = (int)((r[u][q + 2] & 0xFFFFFF00u) | (uint32_t)(q + 2));
+          const int kb1 = (int)((r[u][q + 3] & 0xFFFFFF00u) | (uint32_t)(q + 3));
+          const int alo = min(ka0, ka1), ahi = max(ka0, ka1);
+          const int blo = min(kb0, kb1), bhi = max(kb0, kb1);
+          a2 = __vimin3_s32(max(a1, alo), a2, ahi);
+          a1 = min(a1, alo);
+          b2 = __vimin3_s32(max(b1, blo), b2, bhi);
+          b1 = min(b1, blo);
+        }
+        const int chunk = (cc + u) << 5;
+        const int c1 = min(a1, b1) | chunk, c2 = min(max(a1, b1), min(a2, b2)) | chunk;
+        k2 = min(max(k1, c1), min(k2, c2));
+        k1 = min(k1, c1);
+      }
+    }
+    int code = k1 & 0xFF;
+    const float d1 = __int_as_float(k1 & (int)0xFFFFFF00u);
+    const float d2 = __int_as_float(k2 & (int)0xFFFFFF00u);
+    const bool refine = ok && !(d2 - d1 > 2.f * err + 6.1035156e-5f * d2);
+    if (__any_sync(0xffffffffu, refine)) {
+      // every codeword whose fast distance is within 2 err of the minimum
+      const float thr = d1 * (1.f + 6.1035156e-5f) + 2.f * err;
+      float xe[G];
+#pragma unroll
+      for (int k8 = 0; k8 < G / 8; ++k8) {
+        const uint4 v = *reinterpret_cast<const uint4*>(asmem + core_off<KP>(row, k8));
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) { xe[k8 * 8 + 2 * i] = bf16_lo(w[i]); xe[k8 * 8 + 2 * i + 1] = bf16_hi(w[i]); }
+      }
+      float best = INFINITY;
+      int bi = code;
+#pragma unroll 1
+      for (int cc = 0; cc < kTcCodes / 32; ++cc) {
+        uint32_t r[32];
+        tmem_ld32(t_row + (uint32_t)(cc * 32), r);
+        tmem_wait_ld();
+        uint32_t cand = 0;
+#pragma unroll
+        for (int q = 0; q < 32; ++q) cand |= (__uint_as_float(r[q]) <= thr ? 1u : 0u) << q;
+        if (!refine) cand = 0;
+        while (cand) {
+          const int c = cc * 32 + __ffs(cand) - 1;
+          cand &= cand - 1;
+          float d = 0.f;
+#pragma unroll
+          for (int k8 = 0; k8 < G / 8; ++k8) {
+            const uint4 v = *reinterpret_cast<const uint4*>(bsm + core_off<KP>(c, k8));
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              // B holds -2c: c = -B/2 exactly
+              const float df0 = xe[k8 * 8 + 2 * i] + 0.5f * bf16_lo(w[i]);
+              const float df1 = xe[k8 * 8 + 2 * i + 1] + 0.5f * bf16_hi(w[i]);
+              d = fmaf(df0, df0, d);
+              d = fmaf(df1, df1, d);
+            }
+          }
+          if (d < best) { best = d; bi = c; }
+        }
+      }
+      if (refine) code = bi;
+    }
+    if (ok) p.pool[pool_byte(p.J, p.kind, p.pool_tokens, b, p.H, h, p.tok_off + n, j)] = (uint8_t)code;
+    tmem_fence_before();  // TMEM reads ordered before the next tile's barrier and MMA
+  }
+  __syncthreads();
+  tmem_fence_after();
+  if (warp == 0)
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTcCodes));
+}
+
+template <int G>
+static cudaError_t launch_encode_tc(const EncodeTcParams& p, dim3 grid, cudaStream_t s) {
+  constexpr int KP = ((G + 6) + 15) / 16 * 16;
+  constexpr int need = kTcCodes * KP * 2 + kTcTile * KP * 2 + 64;
+  constexpr int smem = need > kTcSmemFloor ? need : kTcSmemFloor;
+  auto fn = encode_tc_kernel<G, KP>;
+  cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  fn<<<grid, kTcThreads, smem, s>>>(p);
+  return cudaGetLastError();
+}
+
+// Tensor-core path of loopvq_encode: bf16 sub-vectors and 256-entry bf16
+// codebooks with G in {16, 32} and W a multiple of 4.  Returns false (and
+// launches nothing) when the shape is not served.
+bool encode_tc_try(const Geo& g, const void* cb, int kind, const void* x, int64_t n_tokens, int64_t st, int64_t sn,
+                   int64_t sh, uint8_t* pool, int64_t tok_off, int64_t pool_tokens, cudaStream_t s, cudaError_t* err) {
+  if (!g.cb_bf16 || g.C != kTcCodes || (g.G != 16 && g.G != 32) || (g.W & 3)) return false;
+  if (((uintptr_t)x & 7) || (st & 3) || (sn & 3) || (sh & 3)) return false;
+  const int64_t tiles = (n_tokens + kTcTile - 1) / kTcTile;
+  const int64_t ctas_y = (tiles + kTcTilesPerCta - 1) / kTcTilesPerCta;
+  if (ctas_y > 65535 || (int64_t)g.NB * g.H > 65535) return false;
+  EncodeTcParams p;
+  p.x = (const __nv_bfloat16*)x;
+  p.st = st; p.sn = sn; p.sh = sh;
+  p.n_tokens = n_tokens;
+  p.cb = (const __nv_bfloat16*)cb;
+  p.Tc = g.Tc; p.H = g.H; p.J = g.J; p.W = g.W; p.kind = kind;
+  p.pool = pool; p.tok_off = tok_off; p.pool_tokens = pool_tokens;
+  // slot j fastest: the J CTAs of one token chunk run together and share its
+  // sectors in L2
+  dim3 grid(g.J, (unsigned)ctas_y, g.NB * g.H);
+  *err = g.G == 16 ? launch_encode_tc<16>(p, grid, s) : launch_encode_tc<32>(p, grid, s);
+  return true;
+}
+
+}  // namespace loopvq
+
+using namespace loopvq;
+
+extern "C" loopvq_status loopvq_read_encode_faults(uint32_t* bits, int32_t clear, loopvq_stream_t stream) {
+  uint32_t v = 0;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (cudaMemcpyFromSymbolAsync(&v, g_encode_faults, sizeof(v), 0, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return LOOPVQ_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return LOOPVQ_ERR_CUDA;
+  if (clear) {
+    const uint32_t z = 0;
+    if (cudaMemcpyToSymbolAsync(g_encode_faults, &z, sizeof(z), 0, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+        cudaStreamSynchronize(s) != cudaSuccess)
+      return LOOPVQ_ERR_CUDA;
+  }
+  if (bits) *bits = v;
+  return v ? LOOPVQ_ERR_DEVICE_FAULT : LOOPVQ_OK;
+}

@@ -38,7 +38,7 @@ EXPORTED = [
     "loopvq_version", "loopvq_status_string", "loopvq_validate_desc", "loopvq_ctx_split",
     "loopvq_bits_per_element",
     "loopvq_codebook_packed_bytes", "loopvq_codebook_pack", "loopvq_index_pool_bytes",
-    "loopvq_index_pool_pack", "loopvq_index_pool_unpack", "loopvq_encode",
+    "loopvq_index_pool_pack", "loopvq_index_pool_unpack", "loopvq_encode", "loopvq_read_encode_faults",
     "loopvq_decode_workspace_bytes", "loopvq_decode_attn", "loopvq_decode_attn_noalloc",
     "loopvq_read_device_status",
     "loopvq_clear_device_status", "loopvq_dense_decode_workspace_bytes", "loopvq_dense_decode_attn",
@@ -85,6 +85,7 @@ def _load() -> ctypes.CDLL:
         "loopvq_index_pool_pack": (ctypes.c_int, [D, ctypes.c_int, U8P, I64, U8P, I64, I64, P]),
         "loopvq_index_pool_unpack": (ctypes.c_int, [D, ctypes.c_int, U8P, I64, I64, I64, U8P, P]),
         "loopvq_encode": (ctypes.c_int, [D, P, ctypes.c_int, P, ctypes.c_int, I64, I64, I64, I64, U8P, I64, I64, P]),
+        "loopvq_read_encode_faults": (ctypes.c_int, [ctypes.POINTER(ctypes.c_uint32), I32, P]),
         "loopvq_decode_workspace_bytes": (SZ, [D, L]),
         "loopvq_decode_attn": (ctypes.c_int, [D, P, P, L, U8P, U8P, P, P, P, ctypes.c_int, I32, F, P,
                                               ctypes.c_int, P, P, SZ, P]),
@@ -211,6 +212,15 @@ def loopvq_encode(desc, cb_packed, kind, x, n_tokens, stride_t, stride_n, stride
     _check("loopvq_encode", _lib.loopvq_encode(
         ctypes.byref(desc), _ptr(cb_packed), kind, _ptr(x), xd, n_tokens, stride_t, stride_n, stride_h,
         _ptr(idx_pool), tok_off, pool_tokens, _stream(stream)))
+
+
+def loopvq_read_encode_faults(clear=False, stream=None):
+    """Returns (status, fault_bits) of the encoder's device fault word; waits for the stream."""
+    bits = ctypes.c_uint32(0)
+    st = _lib.loopvq_read_encode_faults(ctypes.byref(bits), 1 if clear else 0, _stream(stream))
+    if st not in (LOOPVQ_OK, LOOPVQ_ERR_DEVICE_FAULT):
+        raise LoopVQError("loopvq_read_encode_faults", st)
+    return st, bits.value
 
 
 def loopvq_decode_workspace_bytes(desc, layout) -> int:

@@ -172,3 +172,77 @@ def test_codebook_pack_slices():
     sl = raw[off:off + nbytes].view(np.float32).reshape(4, 3, 256, 16, 4)   # [T][H][C][J][W]
     for t in range(4):
         np.testing.assert_array_equal(sl[t], can[t // 2, :, :, :, t % 2, :].transpose(0, 2, 1, 3))
+
+
+@pytest.mark.parametrize("tc,G", [(4, 16), (4, 32), (2, 16), (1, 16)])
+def test_tensor_core_encode_ragged_all_tokens(tc, G):
+    """bf16 encode of 1000 tokens (7 full 128-row tiles and a ragged one of
+    104) x 2 heads, written at an unaligned pool offset: every code is
+    checked against the oracle, and the pool bytes outside the range stay
+    untouched."""
+    L = _L()
+    T, N, H, D = 4, 1000, 2, 128
+    X = synth.loop_correlated(seed=60 + G + tc, n_loop=T, n_tokens=N, n_heads=H, head_dim=D, n_outlier=4)
+    cb = synth.codebook_from_rows(X, tc, G, 256, seed=61 + G + tc)
+    desc = L.make_desc(T, tc, H, D, G, 256)
+    tok_off, pool_tokens = 37, 1088
+    packed = torch.zeros(L.loopvq_codebook_packed_bytes(desc), dtype=torch.uint8, device="cuda")
+    L.loopvq_codebook_pack(desc, torch.from_numpy(cb).cuda().to(torch.bfloat16), packed)
+    x_dev = torch.from_numpy(np.ascontiguousarray(X, dtype=np.float32)).cuda().to(torch.bfloat16)
+    pool = torch.full((L.loopvq_index_pool_bytes(desc, pool_tokens),), 3, dtype=torch.uint8, device="cuda")
+    L.loopvq_encode(desc, packed, L.LOOPVQ_KEYS, x_dev, N, N * H * D, H * D, D, pool, tok_off, pool_tokens)
+    J = D * tc // G
+    allc = torch.zeros((T // tc, H, pool_tokens, J), dtype=torch.uint8, device="cuda")
+    L.loopvq_index_pool_unpack(desc, L.LOOPVQ_KEYS, pool, 0, pool_tokens, pool_tokens, allc)
+    torch.cuda.synchronize()
+    a = allc.cpu().numpy().astype(np.int64)
+    assert np.all(a[:, :, :tok_off] == 3) and np.all(a[:, :, tok_off + N:] == 3)
+    _accept(X, cb, tc, a[:, :, tok_off:tok_off + N])
+    st, bits = L.loopvq_read_encode_faults(clear=True)
+    assert st == L.LOOPVQ_OK and bits == 0
+
+
+def test_tensor_core_encode_exact_ties_go_to_lowest_index():
+    """Codebooks with duplicated codewords and sub-vectors equal to codewords:
+    the distances tie exactly (and are zero for the equal rows), so the
+    result must be the oracle's lowest index, not a near-tie alternative."""
+    L = _L()
+    T, N, H, D, tc, G = 4, 512, 1, 128, 4, 16
+    X = synth.loop_correlated(seed=70, n_loop=T, n_tokens=N, n_heads=H, head_dim=D)
+    cb = synth.codebook_from_rows(X, tc, G, 256, seed=71)
+    # codeword 200 repeats codeword 10, 255 repeats 0, 7 repeats 6
+    for hi, lo in ((200, 10), (255, 0), (7, 6)):
+        cb[:, :, :, hi] = cb[:, :, :, lo]
+    # tokens 0..63 are exactly codewords 0..63 of their slot
+    W = G // tc
+    Xe = X.copy()
+    for j in range(D // W):
+        for t in range(tc):
+            Xe[t, :64, 0, j * W:(j + 1) * W] = cb[0, 0, j, :64, t, :]
+    desc = L.make_desc(T, tc, H, D, G, 256)
+    g, _ = _encode_gpu(desc, cb, Xe, L.LOOPVQ_KEYS, 512)
+    idx, _, _ = O.encode(Xe, cb, tc)
+    expect = np.arange(64)
+    expect = np.where(expect == 7, 6, expect)   # codeword 7 duplicates 6
+    np.testing.assert_array_equal(idx[0, 0, :64], np.repeat(expect[:, None], D // W, axis=1))
+    np.testing.assert_array_equal(g[0, 0, :64], idx[0, 0, :64])
+    assert _accept(Xe, cb, tc, g) == 0
+
+
+@pytest.mark.parametrize("n", [1, 8, 200])
+@pytest.mark.parametrize("tc,G", [(4, 16), (4, 32), (4, 64), (2, 8), (1, 4)])
+@pytest.mark.parametrize("xdt", ["bf16", "f32"])
+def test_few_token_encode_all_tokens(n, tc, G, xdt):
+    """Few-token encode (fewer than 256 tokens: one warp per token, lanes over
+    codes) across J = 8, 16 and 32 slots, bf16 and fp32 inputs: every code is
+    checked against the oracle."""
+    L = _L()
+    T, H, D = 4, 3, 128
+    X = synth.loop_correlated(seed=80 + n + G, n_loop=T, n_tokens=max(n, 256), n_heads=H, head_dim=D,
+                              n_outlier=4)
+    cb = synth.codebook_from_rows(X, tc, G, 256, seed=81 + G)
+    Xn = np.ascontiguousarray(X[:, :n])
+    desc = L.make_desc(T, tc, H, D, G, 256)
+    g, _ = _encode_gpu(desc, cb, Xn, L.LOOPVQ_VALUES, 256, tok_off=5,
+                       x_dtype=torch.bfloat16 if xdt == "bf16" else torch.float32)
+    _accept(Xn, cb, tc, g)
