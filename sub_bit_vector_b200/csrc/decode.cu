@@ -39,6 +39,9 @@ namespace loopvq {
 constexpr int kNW = 16;                      // consumer warps
 constexpr int kThreads = (kNW + 1) * 32;     // + one producer warp
 constexpr int kStages = 4;
+// With static inputs, chunks a body CTA streams before the previous kernel
+// has finished (the rest follow the dependency).
+constexpr int kPreWaitChunks = 4;
 constexpr int kStageBytes = 32768;
 constexpr int kSplitCap = 4064;              // max body tokens per split, multiple of 32
 // One 64 KB region of 256 rows (one per code) of 64 four-byte columns holds
@@ -181,11 +184,8 @@ __device__ __forceinline__ void score_words(const uint32_t (&w0)[N], const uint3
 // for latency hiding): the sum over its J codes of table column lane + s at
 // step s, i.e. slot (s + lane) mod J, which is the tile's byte order.
 template <int J>
-__device__ __forceinline__ void token_score2(const uint8_t* t0, const uint8_t* t1, int lane, uint32_t lb,
-                                             float& s0, float& s1) {
-  uint32_t w0[J / 4], w1[J / 4];
-  load_tile_words<J>(t0, lane, w0);
-  load_tile_words<J>(t1, lane, w1);
+__device__ __forceinline__ void score_pair(const uint32_t (&w0)[J / 4], const uint32_t (&w1)[J / 4], uint32_t lb,
+                                           float& s0, float& s1) {
   uint64_t a01 = 0, a23 = 0, b01 = 0, b23 = 0;   // packed fp32 pairs, 0 bits = (0, 0)
   score_words(w0, w1, lb, a01, a23, b01, b23, std::make_integer_sequence<int, J / 4>{});
   s0 = sum_f32x2(a01) + sum_f32x2(a23);
@@ -212,11 +212,8 @@ __device__ __forceinline__ void hist_words(const uint32_t (&w0)[N], const uint32
 // Adds this lane's token weights of two tiles into the histogram bins of
 // their codes (same columns as the scores).
 template <int J>
-__device__ __forceinline__ void token_hist2(const uint8_t* t0, const uint8_t* t1, int lane, uint32_t lb,
-                                            uint32_t q0, uint32_t q1) {
-  uint32_t w0[J / 4], w1[J / 4];
-  load_tile_words<J>(t0, lane, w0);
-  load_tile_words<J>(t1, lane, w1);
+__device__ __forceinline__ void hist_pair(const uint32_t (&w0)[J / 4], const uint32_t (&w1)[J / 4], uint32_t lb,
+                                          uint32_t q0, uint32_t q1) {
   hist_words(w0, w1, lb, q0, q1, std::make_integer_sequence<int, J / 4>{});
 }
 
@@ -259,30 +256,70 @@ __device__ __forceinline__ float load_q(const void* q, int q_bf16, size_t i) {
 __device__ __forceinline__ void combine_staged(const float* part, int n_splits, int D, void* out, int out_bf16,
                                                float* lse, float* sm, int cap, int tid, int nthr) {
   const int row = D + 4;
-  if (n_splits * row > cap) {
+  const int n4 = n_splits * row / 4;  // rows are 16-byte multiples
+  if (n_splits * row + n_splits > cap || n4 > 4 * nthr || n_splits > 64) {
     combine_splits(part, n_splits, D, out, out_bf16, lse, sm, tid, nthr, ConsumerSync{});
     return;
   }
-  for (int i = tid; i < n_splits * row; i += nthr) sm[i] = __ldcg(part + i);
-  consumer_sync();
-  float M = -INFINITY;
-  for (int s = 0; s < n_splits; ++s) M = fmaxf(M, sm[s * row + D]);
-  float L = 0.f;
-  for (int s = 0; s < n_splits; ++s)
-    if (sm[s * row + D] != -INFINITY) L += sm[s * row + D + 1] * exp2f(sm[s * row + D] - M);
-  if (tid < D) {
-    float o = 0.f;
-    if (M != -INFINITY) {
-      for (int s = 0; s < n_splits; ++s)
-        if (sm[s * row + D] != -INFINITY) o = fmaf(sm[s * row + tid], exp2f(sm[s * row + D] - M), o);
-      o = L > 0.f ? o / L : 0.f;
-    }
-    if (out_bf16)
-      ((__nv_bfloat16*)out)[tid] = __float2bfloat16_rn(o);
-    else
-      ((float*)out)[tid] = o;
+  // every partial in flight at once: one round trip to L2
+  const float4* src = reinterpret_cast<const float4*>(part);
+  float4 v[4];
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const int i = tid + u * nthr;
+    if (i < n4) v[u] = __ldcg(src + i);
   }
-  if (lse && tid == 0) *lse = (M == -INFINITY || !(L > 0.f)) ? -INFINITY : (M + log2f(L)) * 0.6931471805599453f;
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const int i = tid + u * nthr;
+    if (i < n4) reinterpret_cast<float4*>(sm)[i] = v[u];
+  }
+  consumer_sync();
+  // warp 0: the merge weights 2^(m_s - M) / L of every split (lane s, s + 32)
+  float* wgt = sm + n_splits * row;
+  if (tid < 32) {
+    float ms[2], ls[2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int s = tid + 32 * u;
+      ms[u] = s < n_splits ? sm[s * row + D] : -INFINITY;
+      ls[u] = s < n_splits ? sm[s * row + D + 1] : 0.f;
+    }
+    float M = fmaxf(ms[0], ms[1]);
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    float e[2], L = 0.f;
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      e[u] = ms[u] == -INFINITY ? 0.f : exp2f(ms[u] - M);
+      L = fmaf(ls[u], e[u], L);
+    }
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+    const bool ok = M != -INFINITY && L > 0.f;
+    const float inv = ok ? 1.f / L : 0.f;
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int s = tid + 32 * u;
+      if (s < n_splits) wgt[s] = e[u] * inv;
+    }
+    if (lse && tid == 0) *lse = ok ? (M + log2f(L)) * 0.6931471805599453f : -INFINITY;
+  }
+  consumer_sync();
+  if (tid < D) {
+    float o[4] = {0.f, 0.f, 0.f, 0.f};
+    int s = 0;
+    for (; s + 4 <= n_splits; s += 4) {
+#pragma unroll
+      for (int u = 0; u < 4; ++u) o[u] = fmaf(sm[(s + u) * row + tid], wgt[s + u], o[u]);
+    }
+    for (; s < n_splits; ++s) o[0] = fmaf(sm[s * row + tid], wgt[s], o[0]);
+    const float r = (o[0] + o[1]) + (o[2] + o[3]);
+    if (out_bf16)
+      ((__nv_bfloat16*)out)[tid] = __float2bfloat16_rn(r);
+    else
+      ((float*)out)[tid] = r;
+  }
 }
 
 template <int J, int D, typename CBT>
@@ -303,6 +340,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
   const int64_t body_off = __ldg(p.body_off + r);
   const int64_t win_off = __ldg(p.win_off + r);
   const size_t unit = (size_t)r * p.Hq + hq;
+  // The query row is read right after the dependency resolves; pulling its
+  // lines into L2 now (a hint: L2 stays coherent with the previous kernel's
+  // writes) takes the DRAM latency off that critical step.
+  if (p.static_inputs && tid < (D * (p.q_bf16 ? 2 : 4)) / 128) {
+    const char* qrow = reinterpret_cast<const char*>(p.q) + unit * D * (p.q_bf16 ? 2 : 4);
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(qrow + tid * 128));
+  }
   float wk[kPer][W];               // B^K_t entries (c, j) = tid + 512k, code-major slice
   const CBT* bk = reinterpret_cast<const CBT*>(p.cbK_slice) + (size_t)h * p.C * J * W;
   if (tid < kNW * 32) {
@@ -405,6 +449,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
       const int n_slice = (is_window || n_tok == 0) ? 0 : (int)((vslice_bytes + kStageBytes - 1) / kStageBytes);
       for (int k = 0; k < n_chunks + n_slice; ++k) {
         const int s = k % kStages;
+        if (k == kPreWaitChunks && p.static_inputs && !is_window) griddep_wait();
         if (k >= kStages) {
           if (!mbar_wait_bounded(smem_u32(empty_bar + s), ((k / kStages) - 1) & 1)) {
             set_fault(p.status, LOOPVQ_FAULT_TIMEOUT);
@@ -562,6 +607,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
     const uint32_t lb = region | (uint32_t)(lane * 4);
     consumer_sync();
 
+    // Each warp owns tiles warp + kNW*i (i < kTPW) of every chunk.  It copies
+    // their code words (16 per lane) to registers and releases the stage at
+    // once, so the producer refills it while the warp gathers.
+    constexpr int kTPW = kTilesPerChunk / kNW;  // 2, 4, 8 for J = 32, 16, 8
+    constexpr int kWPT = J / 4;                 // code words per tile and lane
+
     // ---- pass K: scores and split maximum
     float mx = -INFINITY;
     bool nan_seen = false;
@@ -570,25 +621,34 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
       if (!mbar_wait_bounded(smem_u32(full_bar + s), (k / kStages) & 1)) set_fault(p.status, LOOPVQ_FAULT_TIMEOUT);
       const uint8_t* st = stage_ptr(s);
       const int nt = min(kTilesPerChunk, n_tiles - k * kTilesPerChunk);
-      for (int tl = warp; tl < nt; tl += 2 * kNW) {
-        const int tl2 = tl + kNW < nt ? tl + kNW : tl;
-        float sv0, sv1;
-        token_score2<J>(st + tl * 32 * J, st + tl2 * 32 * J, lane, lb, sv0, sv1);
-        const int tok0c = (k * kTilesPerChunk + tl) * 32 + lane;
-        const bool v0 = tok0c < n_tok;
-        if (v0 && sv0 != sv0) nan_seen = true;
-        sc[tok0c] = v0 ? sv0 : -INFINITY;
-        mx = fmaxf(mx, v0 ? sv0 : -INFINITY);
-        if (tl2 != tl) {
-          const int tok1c = (k * kTilesPerChunk + tl2) * 32 + lane;
-          const bool v1 = tok1c < n_tok;
-          if (v1 && sv1 != sv1) nan_seen = true;
-          sc[tok1c] = v1 ? sv1 : -INFINITY;
-          mx = fmaxf(mx, v1 ? sv1 : -INFINITY);
+      uint32_t wd[kTPW][kWPT];
+#pragma unroll
+      for (int i = 0; i < kTPW; ++i) {
+        if (warp + kNW * i < nt) {
+          load_tile_words<J>(st + (warp + kNW * i) * 32 * J, lane, wd[i]);
+        } else {
+#pragma unroll
+          for (int x = 0; x < kWPT; ++x) wd[i][x] = 0u;
         }
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(empty_bar + s));
+#pragma unroll
+      for (int i = 0; i < kTPW; i += 2) {
+        const int tl = warp + kNW * i;
+        if (tl < nt) {
+          float sv[2];
+          score_pair<J>(wd[i], wd[i + 1], lb, sv[0], sv[1]);
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const int tok = (k * kTilesPerChunk + tl + kNW * u) * 32 + lane;
+            const bool v = (tl + kNW * u < nt) && tok < n_tok;
+            if (v && sv[u] != sv[u]) nan_seen = true;
+            if (tl + kNW * u < nt) sc[tok] = v ? sv[u] : -INFINITY;
+            mx = fmaxf(mx, v ? sv[u] : -INFINITY);
+          }
+        }
+      }
     }
     if (nan_seen) set_fault(p.status, LOOPVQ_FAULT_CODE_RANGE);
 #pragma unroll
@@ -612,42 +672,46 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
       const uint8_t* st = stage_ptr(s);
       const int kv = k - n_chunks_half;
       const int nt = min(kTilesPerChunk, n_tiles - kv * kTilesPerChunk);
-      for (int tl = warp; tl < nt; tl += 2 * kNW) {
-        const int tl2 = tl + kNW < nt ? tl + kNW : tl;
-        uint32_t qv[2];
+      uint32_t wd[kTPW][kWPT];
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          const int tok = (kv * kTilesPerChunk + (u ? tl2 : tl)) * 32 + lane;
-          qv[u] = 0;
-          if (tok < n_tok && (u == 0 || tl2 != tl)) {
-            const float pw = exp2f(sc[tok] - m);
-            const uint32_t seq = (uint32_t)(body_off + tok0 + tok);
-            const float uu = (float)((seq * 2654435769u) >> 8) * (1.0f / 16777216.0f);
-            qv[u] = __float2uint_rd(fmaf(pw, scaleS, uu));
-          }
-          qsum += qv[u];
+      for (int i = 0; i < kTPW; ++i) {
+        if (warp + kNW * i < nt) {
+          load_tile_words<J>(st + (warp + kNW * i) * 32 * J, lane, wd[i]);
+        } else {
+#pragma unroll
+          for (int x = 0; x < kWPT; ++x) wd[i][x] = 0u;
         }
-        token_hist2<J>(st + tl * 32 * J, st + tl2 * 32 * J, lane, lb, qv[0], qv[1]);
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(empty_bar + s));
+#pragma unroll
+      for (int i = 0; i < kTPW; i += 2) {
+        const int tl = warp + kNW * i;
+        if (tl < nt) {
+          uint32_t qv[2];
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const int tok = (kv * kTilesPerChunk + tl + kNW * u) * 32 + lane;
+            qv[u] = 0;
+            if (tl + kNW * u < nt && tok < n_tok) {
+              const float pw = exp2f(sc[tok] - m);
+              const uint32_t seq = (uint32_t)(body_off + tok0 + tok);
+              const float uu = (float)((seq * 2654435769u) >> 8) * (1.0f / 16777216.0f);
+              qv[u] = __float2uint_rd(fmaf(pw, scaleS, uu));
+            }
+            qsum += qv[u];
+          }
+          hist_pair<J>(wd[i], wd[i + 1], lb, qv[0], qv[1]);
+        }
+      }
     }
-    // epilogue operands: entries (c, j) = ctid + 512k of the code-major value
-    // slice, which the producer bulk-copied into the drained ring stages
+    // the value codebook slice (code-major entries (c, j) = ctid + 512k),
+    // which the producer bulk-copied into the drained ring stages
     const int n_slice = (n_tok == 0) ? 0 : (int)((p.C * D * sizeof(CBT) + kStageBytes - 1) / kStageBytes);
     for (int i = 0; i < n_slice; ++i) {
       const int k = n_chunks + i;
       if (!mbar_wait_bounded(smem_u32(full_bar + (k % kStages)), (k / kStages) & 1))
         set_fault(p.status, LOOPVQ_FAULT_TIMEOUT);
-    }
-    float vv[kPer][W];
-#pragma unroll
-    for (int k = 0; k < kPer; ++k) {
-      const int e = ctid + k * kNW * 32;
-      const uint32_t off = (uint32_t)e * W * sizeof(CBT);
-      const CBT* src = reinterpret_cast<const CBT*>(stage_ptr((n_chunks + (int)(off / kStageBytes)) % kStages) +
-                                                    off % kStageBytes);
-      load_vec<W>(src, n_slice > 0 && e / J < p.C, vv[k]);
     }
 #pragma unroll
     for (int o = 16; o >= 1; o >>= 1) qsum += __shfl_xor_sync(0xffffffffu, qsum, o);
@@ -657,23 +721,31 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
     // ---- epilogue: o[d] = 2^-S sum_c hist[j][c] B^V_t[c][j][w].  Thread
     // ctid accumulates its W outputs over entries (c, j) = ctid + 512k; the
     // 512/J partial groups per output are summed through shared memory (the
-    // LUT region is free by now).
+    // score buffer is free by now).
     {
-      float acc[W];
-#pragma unroll
-      for (int w = 0; w < W; ++w) acc[w] = 0.f;
       const int j = ctid % J;
+      float hf[kPer];
 #pragma unroll
       for (int k = 0; k < kPer; ++k) {
         const int c = (ctid + k * kNW * 32) / J;
         uint32_t hs = 0;
 #pragma unroll
         for (int g = 0; g < kCols / J; ++g) hs += hist[c * kCols + g * J + j];
-        if (c < p.C && hs != 0u) {
-          const float hf = (float)hs;
+        hf[k] = c < p.C ? (float)hs : 0.f;
+      }
+      float acc[W];
 #pragma unroll
-          for (int w = 0; w < W; ++w) acc[w] = fmaf(hf, vv[k][w], acc[w]);
-        }
+      for (int w = 0; w < W; ++w) acc[w] = 0.f;
+#pragma unroll
+      for (int k = 0; k < kPer; ++k) {
+        const int e = ctid + k * kNW * 32;
+        const uint32_t off = (uint32_t)e * W * sizeof(CBT);
+        const CBT* src = reinterpret_cast<const CBT*>(stage_ptr((n_chunks + (int)(off / kStageBytes)) % kStages) +
+                                                      off % kStageBytes);
+        float vv[W];
+        load_vec<W>(src, n_slice > 0 && e / J < p.C, vv);
+#pragma unroll
+        for (int w = 0; w < W; ++w) acc[w] = fmaf(hf[k], vv[w], acc[w]);
       }
       // bins of codes >= n_codes must be empty
       if (p.C < 256) {
@@ -689,32 +761,39 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
       }
       float* ored = sc;  // [kNW][D] per-warp partial sums; scores are no longer read
       if (lane < J) {
+        if constexpr (W % 4 == 0) {
 #pragma unroll
-        for (int w = 0; w < W; ++w) ored[warp * D + j * W + w] = acc[w];
+          for (int w = 0; w < W; w += 4)
+            *reinterpret_cast<float4*>(ored + warp * D + j * W + w) = make_float4(acc[w], acc[w + 1], acc[w + 2], acc[w + 3]);
+        } else {
+#pragma unroll
+          for (int w = 0; w < W; ++w) ored[warp * D + j * W + w] = acc[w];
+        }
       }
       consumer_sync();
       if (ctid < D) {
         float o = 0.f;
 #pragma unroll
         for (int i = 0; i < kNW; ++i) o += ored[i * D + ctid];
-        part[ctid] = o / scaleS;
+        part[ctid] = o * (1.f / scaleS);  // exact: a power of two
       }
     }
     if (ctid == 0) {
       uint64_t tot = 0;
       for (int w = 0; w < kNW; ++w) tot += reinterpret_cast<uint32_t*>(red)[kNW + w];
       part[D] = m;
-      part[D + 1] = (float)tot / scaleS;
+      part[D + 1] = (float)tot * (1.f / scaleS);
     }
   }
 
   // ---- split ticket and combine -------------------------------------------
   consumer_sync();
   if (ctid == 0) {
-    __threadfence();
-    const uint32_t t = atomicAdd(p.tickets + unit, 1u);
-    __threadfence();
-    *flag = (t == (uint32_t)(n_splits - 1)) ? 1 : 0;
+    // release: this CTA's partial (ordered before by the barrier) before the
+    // ticket; acquire: the other splits' partials after theirs
+    uint32_t t;
+    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(t) : "l"(p.tickets + unit) : "memory");
+    *flag = t == (uint32_t)(n_splits - 1);
   }
   consumer_sync();
   if (*flag) {
