@@ -257,7 +257,7 @@ __device__ __forceinline__ void combine_staged(const float* part, int n_splits, 
                                                float* lse, float* sm, int cap, int tid, int nthr) {
   const int row = D + 4;
   const int n4 = n_splits * row / 4;  // rows are 16-byte multiples
-  if (n_splits * row + n_splits > cap || n4 > 4 * nthr || n_splits > 64) {
+  if (n_splits * row > cap || n4 > 4 * nthr || n_splits > 64) {
     combine_splits(part, n_splits, D, out, out_bf16, lse, sm, tid, nthr, ConsumerSync{});
     return;
   }
@@ -275,13 +275,14 @@ __device__ __forceinline__ void combine_staged(const float* part, int n_splits, 
     if (i < n4) reinterpret_cast<float4*>(sm)[i] = v[u];
   }
   consumer_sync();
-  // warp 0: the merge weights 2^(m_s - M) / L of every split (lane s, s + 32)
-  float* wgt = sm + n_splits * row;
-  if (tid < 32) {
+  // Each warp that writes outputs derives the merge weights 2^(m_s - M) / L
+  // itself (lane s holds splits s and s + 32), so no second barrier.
+  if (tid < D) {
+    const int lane = tid & 31;
     float ms[2], ls[2];
 #pragma unroll
     for (int u = 0; u < 2; ++u) {
-      const int s = tid + 32 * u;
+      const int s = lane + 32 * u;
       ms[u] = s < n_splits ? sm[s * row + D] : -INFINITY;
       ls[u] = s < n_splits ? sm[s * row + D + 1] : 0.f;
     }
@@ -297,28 +298,18 @@ __device__ __forceinline__ void combine_staged(const float* part, int n_splits, 
 #pragma unroll
     for (int o = 16; o >= 1; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
     const bool ok = M != -INFINITY && L > 0.f;
-    const float inv = ok ? 1.f / L : 0.f;
-#pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      const int s = tid + 32 * u;
-      if (s < n_splits) wgt[s] = e[u] * inv;
-    }
-    if (lse && tid == 0) *lse = ok ? (M + log2f(L)) * 0.6931471805599453f : -INFINITY;
-  }
-  consumer_sync();
-  if (tid < D) {
-    float o[4] = {0.f, 0.f, 0.f, 0.f};
-    int s = 0;
-    for (; s + 4 <= n_splits; s += 4) {
-#pragma unroll
-      for (int u = 0; u < 4; ++u) o[u] = fmaf(sm[(s + u) * row + tid], wgt[s + u], o[u]);
-    }
-    for (; s < n_splits; ++s) o[0] = fmaf(sm[s * row + tid], wgt[s], o[0]);
-    const float r = (o[0] + o[1]) + (o[2] + o[3]);
+    const float inv = ok ? __frcp_rn(L) : 0.f;
+    const float w0 = e[0] * inv, w1 = e[1] * inv;
+    float o4[4] = {0.f, 0.f, 0.f, 0.f};
+    const int n0 = n_splits < 32 ? n_splits : 32;
+    for (int s = 0; s < n0; ++s) o4[s & 3] = fmaf(sm[s * row + tid], __shfl_sync(0xffffffffu, w0, s), o4[s & 3]);
+    for (int s = 32; s < n_splits; ++s) o4[s & 3] = fmaf(sm[s * row + tid], __shfl_sync(0xffffffffu, w1, s - 32), o4[s & 3]);
+    const float r = (o4[0] + o4[1]) + (o4[2] + o4[3]);
     if (out_bf16)
       ((__nv_bfloat16*)out)[tid] = __float2bfloat16_rn(r);
     else
       ((float*)out)[tid] = r;
+    if (lse && tid == 0) *lse = ok ? (M + log2f(L)) * 0.6931471805599453f : -INFINITY;
   }
 }
 
