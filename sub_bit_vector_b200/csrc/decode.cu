@@ -317,7 +317,10 @@ template <int J, int D, typename CBT>
 __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams p) {
   extern __shared__ __align__(1024) uint8_t dyn[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int split = blockIdx.x, hq = blockIdx.y, r = blockIdx.z;
+  // Query head fastest, the window split last: CTAs are dispatched in this
+  // order, so the light window splits take the SMs that the previous launch
+  // frees last and every body split starts (and prefetches) as early as it can.
+  const int hq = blockIdx.x, split = blockIdx.y, r = blockIdx.z;
   const int group = p.Hq / p.H;
   const int h = hq / group;
   constexpr int W = D / J;
@@ -371,8 +374,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
     return;
   }
   if (split >= n_splits) return;
-  const bool is_window = split < has_win;
-  const int bsplit = split - has_win;
+  const bool is_window = has_win && split == n_body_splits;  // partial row n_body_splits
+  const int bsplit = split;
   if (is_window) {
     if (win_off < 0 || win_off + n_win > p.win_pool_tokens) bad = true;
   } else {
@@ -930,7 +933,7 @@ extern "C" loopvq_status loopvq_decode_attn(const loopvq_codebook_desc* desc, co
 
   p.static_inputs = (layout->flags & LOOPVQ_LAYOUT_STATIC_INPUTS) ? 1 : 0;
 
-  dim3 grid(pl.max_splits, g.Hq, layout->batch);
+  dim3 grid(g.Hq, pl.max_splits, layout->batch);
   cudaStream_t s = (cudaStream_t)stream;
 #define LOOPVQ_LAUNCH(JJ, DD, CBT)                                                                    \
   do {                                                                                               \
@@ -1066,7 +1069,7 @@ extern "C" loopvq_status loopvq_decode_attn_noalloc(const loopvq_codebook_desc* 
 
   p.static_inputs = (layout->flags & LOOPVQ_LAYOUT_STATIC_INPUTS) ? 1 : 0;
 
-  dim3 grid(pl.max_splits, g.Hq, layout->batch);
+  dim3 grid(g.Hq, pl.max_splits, layout->batch);
 #define LOOPVQ_LAUNCH(JJ, DD, CBT)                                                                    \
   do {                                                                                               \
     auto kfn = decode_kernel<JJ, DD, CBT>;                                                           \
