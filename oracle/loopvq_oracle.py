@@ -61,6 +61,9 @@ __all__ = [
     "decode_attention",
     "dense_decode_attention",
     "reconstruction_mse",
+    "kmeans_update",
+    "kmeans",
+    "distortion",
 ]
 
 
@@ -330,3 +333,70 @@ def reconstruction_mse(X: np.ndarray, idx: np.ndarray, codebook: np.ndarray, tc:
         acc += float(np.sum(diff * diff))
         count += diff.size
     return acc / count
+
+
+# --------------------------------------------------------------------------
+# codebook construction (Lloyd's k-means on the loop-axis sub-vectors)
+# --------------------------------------------------------------------------
+# The pages fine-tune codebooks against the full-precision model and do not
+# say where the fine-tuning starts.  The plain data-driven start is Lloyd's
+# k-means on the same loop-axis sub-vectors the encoder codes, seeded from
+# data rows: alternate the nearest-codeword assignment (``encode``) with the
+# update below.
+
+def kmeans_update(X: np.ndarray, idx: np.ndarray, codebook: np.ndarray, tc: int):
+    """One Lloyd update of every codebook, by definition.
+
+    Codeword c of (block b, head h, slot j) becomes the mean of the
+    sub-vectors (``form_subvectors``) of the tokens whose code ``idx[b][h][n][j]``
+    is c; a codeword that no token uses keeps its value.  Returns
+    ``(new_codebook, counts)``: the codebook in fp64, same layout
+    ``[NB][H][J][C][Tc][W]``, and the member counts ``[NB][H][J][C]``.
+    """
+    NB, H, J, C, tc2, w = codebook.shape
+    if tc2 != tc:
+        raise ValueError("codebook Tc does not match")
+    new = np.array(codebook, dtype=np.float64).reshape(NB, H, J, C, tc * w)
+    counts = np.zeros((NB, H, J, C), dtype=np.int64)
+    for b in range(NB):
+        sub = form_subvectors(X, b, tc, w)  # [N][H][J][G]
+        for h in range(H):
+            for j in range(J):
+                codes = np.asarray(idx[b, h, :, j], dtype=np.int64)
+                for c in np.unique(codes):
+                    members = sub[codes == c, h, j]
+                    new[b, h, j, c] = members.sum(axis=0) / len(members)
+                    counts[b, h, j, c] = len(members)
+    return new.reshape(NB, H, J, C, tc, w), counts
+
+
+def distortion(X: np.ndarray, idx: np.ndarray, codebook: np.ndarray, tc: int) -> float:
+    """Sum over all sub-vectors of the squared distance to their codeword."""
+    NB, H, J, C, tc2, w = codebook.shape
+    cb = np.asarray(codebook, dtype=np.float64).reshape(NB, H, J, C, tc * w)
+    total = 0.0
+    for b in range(NB):
+        sub = form_subvectors(X, b, tc, w)
+        for h in range(H):
+            for j in range(J):
+                diff = sub[:, h, j] - cb[b, h, j, idx[b, h, :, j]]
+                total += float(np.sum(diff * diff))
+    return total
+
+
+def kmeans(X: np.ndarray, codebook: np.ndarray, tc: int, n_iter: int):
+    """Lloyd's algorithm from ``codebook``: ``n_iter`` rounds of nearest-codeword
+    assignment (``encode``, ties to the lowest index) then ``kmeans_update``.
+
+    Returns ``(codebook, idx, history)`` where ``history[i]`` is the
+    distortion of round i's assignment against the codebook it was made
+    with (non-increasing in i).
+    """
+    cb = np.asarray(codebook, dtype=np.float64)
+    history = []
+    idx = None
+    for _ in range(n_iter):
+        idx, _, _ = encode(X, cb, tc)
+        history.append(distortion(X, idx, cb, tc))
+        cb, _ = kmeans_update(X, idx, cb, tc)
+    return cb, idx, history

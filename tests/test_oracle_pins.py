@@ -328,3 +328,87 @@ def test_generator_loop_correlation_and_scale():
     per_chan = np.abs(K).mean(axis=(0, 1))           # [H][D]
     assert np.all(np.sort(per_chan, axis=1)[:, -4:].min(axis=1) > 3 * np.median(per_chan))
     assert np.array_equal(K, synth.round_bf16(K))    # already bf16 values
+
+
+# ---------------------------------------------------------- codebook k-means
+
+def _small_kv(seed, n=600, h=2, d=16):
+    return synth.loop_correlated(seed=seed, n_loop=4, n_tokens=n, n_heads=h, head_dim=d, n_outlier=1)
+
+
+def test_kmeans_one_round_matches_scikit_learn_lloyd():
+    """One Lloyd round (nearest-codeword assignment, then means) against
+    scikit-learn's Lloyd k-means started from the same centers; the codebook
+    is made of data rows, so no cluster is empty."""
+    from sklearn.cluster import KMeans
+    X = _small_kv(500)
+    tc, G, C = 4, 16, 32
+    cb = synth.codebook_from_rows(X, tc, G, C, seed=501)
+    new, idx, _ = O.kmeans(X, cb, tc, 1)
+    W = G // tc
+    sub = O.form_subvectors(X, 0, tc, W)
+    for h in range(X.shape[2]):
+        for j in range(X.shape[3] // W):
+            init = cb[0, h, j].reshape(C, G).astype(np.float64)
+            km = KMeans(n_clusters=C, init=init, n_init=1, max_iter=1, tol=0.0, algorithm="lloyd")
+            km.fit(sub[:, h, j])
+            np.testing.assert_allclose(new[0, h, j].reshape(C, G), km.cluster_centers_, rtol=1e-12, atol=1e-12)
+
+
+def test_kmeans_update_single_member_and_empty_cluster():
+    """A codeword with one member becomes that sub-vector exactly; a codeword
+    without members keeps its value."""
+    X = _small_kv(510, n=8, h=1, d=8)
+    tc, G = 4, 8  # W = 2, J = 4
+    rng = np.random.default_rng(511)
+    cb = rng.standard_normal((1, 1, 4, 16, tc, G // tc))
+    idx = np.zeros((1, 1, 8, 4), dtype=np.int64)
+    idx[0, 0, :, :] = np.arange(8)[:, None]          # token n -> code n in every slot
+    new, counts = O.kmeans_update(X, idx, cb, tc)
+    sub = O.form_subvectors(X, 0, tc, G // tc)
+    for j in range(4):
+        for n in range(8):
+            np.testing.assert_array_equal(new[0, 0, j, n].reshape(-1), sub[n, 0, j])
+        np.testing.assert_array_equal(new[0, 0, j, 8:], cb[0, 0, j, 8:])
+        assert list(counts[0, 0, j]) == [1] * 8 + [0] * 8
+
+
+def test_kmeans_update_closed_form_two_clusters():
+    """Two hand-made groups of sub-vectors: the update is their arithmetic
+    means, written out."""
+    X = np.zeros((1, 5, 1, 2))
+    X[0, :, 0, 0] = [1.0, 2.0, 3.0, 10.0, 14.0]
+    X[0, :, 0, 1] = [0.0, 0.0, 3.0, -2.0, -4.0]
+    cb = np.zeros((1, 1, 1, 2, 1, 2))
+    idx = np.array([0, 0, 0, 1, 1]).reshape(1, 1, 5, 1)
+    new, counts = O.kmeans_update(X, idx, cb, 1)
+    np.testing.assert_allclose(new[0, 0, 0, 0, 0], [2.0, 1.0])
+    np.testing.assert_allclose(new[0, 0, 0, 1, 0], [12.0, -3.0])
+    assert list(counts[0, 0, 0]) == [3, 2]
+
+
+def test_kmeans_update_is_the_distortion_minimiser_and_a_fixed_point():
+    """For a fixed assignment the mean minimises the squared error: any
+    perturbation of the updated codebook raises the distortion; updating
+    again with the same assignment changes nothing."""
+    X = _small_kv(520)
+    tc, G, C = 2, 8, 16
+    cb = synth.codebook_from_rows(X, tc, G, C, seed=521)
+    idx, _, _ = O.encode(X, cb, tc)
+    new, _ = O.kmeans_update(X, idx, cb, tc)
+    base = O.distortion(X, idx, new, tc)
+    assert base <= O.distortion(X, idx, cb, tc)
+    rng = np.random.default_rng(522)
+    for _ in range(3):
+        bumped = new + 1e-3 * rng.standard_normal(new.shape)
+        assert O.distortion(X, idx, bumped, tc) > base
+    again, _ = O.kmeans_update(X, idx, new, tc)
+    np.testing.assert_allclose(again, new, rtol=0, atol=1e-13)
+
+
+def test_lloyd_distortion_never_increases():
+    X = _small_kv(530)
+    cb = synth.codebook_from_rows(X, 4, 16, 32, seed=531)
+    _, _, hist = O.kmeans(X, cb, 4, 5)
+    assert all(b <= a * (1 + 1e-12) for a, b in zip(hist, hist[1:]))
+    assert hist[-1] < hist[0]
