@@ -240,6 +240,38 @@ LOOPVQ_API loopvq_status loopvq_encode(const loopvq_codebook_desc* desc, const v
  * clear != 0 zeroes the word afterwards. */
 LOOPVQ_API loopvq_status loopvq_read_encode_faults(uint32_t* bits, int32_t clear, loopvq_stream_t stream);
 
+/* ------------------------------------------------ codebook construction */
+
+/*
+ * One Lloyd (k-means) update of every codebook.  Project page, "Method" --
+ * "Loop-aware codebook fine-tuning": the codebooks are fine-tuned against the
+ * full-precision model from a start the pages do not state; the data-driven
+ * start is k-means on the loop-axis sub-vectors, i.e. rounds of
+ * loopvq_encode (nearest-codeword assignment) followed by this call.
+ * Codeword c of (block b, head h, slot j) becomes the mean, in fp32, of the
+ * sub-vectors of the n_tokens tokens whose stored code is c; a codeword no
+ * token uses keeps its value from cb_in.  Codes >= n_codes are ignored.
+ *   x, x_dtype, n_tokens, strides : as in loopvq_encode.
+ *   kind, idx_pool, tok_off, pool_tokens : where loopvq_encode wrote the
+ *               codes of these tokens (token n at pool position tok_off + n).
+ *   cb_in, cb_out : device, CANONICAL layout [NB][H][J][C][Tc][W] in
+ *               desc->cb_dtype (bf16 output is rounded to nearest); must not
+ *               alias.  Re-pack cb_out with loopvq_codebook_pack before
+ *               encoding or decoding with it.
+ *   counts_out : device int32 [NB][H][J][C] member counts, or NULL.
+ *   workspace  : device, 256-byte aligned, at least
+ *               loopvq_codebook_update_workspace_bytes(desc) bytes; the call
+ *               zeroes it on the stream.
+ * Sums use fp32 atomics, so results are reproducible only up to rounding.
+ */
+LOOPVQ_API size_t loopvq_codebook_update_workspace_bytes(const loopvq_codebook_desc* desc);
+LOOPVQ_API loopvq_status loopvq_codebook_update(const loopvq_codebook_desc* desc, loopvq_kind kind,
+                                                const void* x, loopvq_dtype x_dtype, int64_t n_tokens,
+                                                int64_t stride_t, int64_t stride_n, int64_t stride_h,
+                                                const uint8_t* idx_pool, int64_t tok_off, int64_t pool_tokens,
+                                                const void* cb_in, void* cb_out, int32_t* counts_out,
+                                                void* workspace, size_t workspace_bytes, loopvq_stream_t stream);
+
 /* ---------------------------------------------------------------- decode */
 
 /* Workspace bytes loopvq_decode_attn needs for this layout (0 if invalid). */

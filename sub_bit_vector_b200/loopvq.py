@@ -39,6 +39,7 @@ EXPORTED = [
     "loopvq_bits_per_element",
     "loopvq_codebook_packed_bytes", "loopvq_codebook_pack", "loopvq_index_pool_bytes",
     "loopvq_index_pool_pack", "loopvq_index_pool_unpack", "loopvq_encode", "loopvq_read_encode_faults",
+    "loopvq_codebook_update_workspace_bytes", "loopvq_codebook_update",
     "loopvq_decode_workspace_bytes", "loopvq_decode_attn", "loopvq_decode_attn_noalloc",
     "loopvq_read_device_status",
     "loopvq_clear_device_status", "loopvq_dense_decode_workspace_bytes", "loopvq_dense_decode_attn",
@@ -86,6 +87,9 @@ def _load() -> ctypes.CDLL:
         "loopvq_index_pool_unpack": (ctypes.c_int, [D, ctypes.c_int, U8P, I64, I64, I64, U8P, P]),
         "loopvq_encode": (ctypes.c_int, [D, P, ctypes.c_int, P, ctypes.c_int, I64, I64, I64, I64, U8P, I64, I64, P]),
         "loopvq_read_encode_faults": (ctypes.c_int, [ctypes.POINTER(ctypes.c_uint32), I32, P]),
+        "loopvq_codebook_update_workspace_bytes": (SZ, [D]),
+        "loopvq_codebook_update": (ctypes.c_int, [D, ctypes.c_int, P, ctypes.c_int, I64, I64, I64, I64, U8P, I64, I64,
+                                                  P, P, P, P, SZ, P]),
         "loopvq_decode_workspace_bytes": (SZ, [D, L]),
         "loopvq_decode_attn": (ctypes.c_int, [D, P, P, L, U8P, U8P, P, P, P, ctypes.c_int, I32, F, P,
                                               ctypes.c_int, P, P, SZ, P]),
@@ -133,6 +137,10 @@ def _stream(stream) -> Optional[int]:
     if isinstance(stream, int):
         return stream
     return stream.cuda_stream
+
+
+def _nbytes(t) -> int:
+    return t.numel() * t.element_size()
 
 
 def _dtype_code(t) -> int:
@@ -221,6 +229,19 @@ def loopvq_read_encode_faults(clear=False, stream=None):
     if st not in (LOOPVQ_OK, LOOPVQ_ERR_DEVICE_FAULT):
         raise LoopVQError("loopvq_read_encode_faults", st)
     return st, bits.value
+
+
+def loopvq_codebook_update_workspace_bytes(desc) -> int:
+    return _lib.loopvq_codebook_update_workspace_bytes(ctypes.byref(desc))
+
+
+def loopvq_codebook_update(desc, kind, x, n_tokens, stride_t, stride_n, stride_h, idx_pool, tok_off, pool_tokens,
+                           cb_in, cb_out, counts_out, workspace, stream=None, x_dtype=None) -> None:
+    xd = _dtype_code(x) if x_dtype is None else x_dtype
+    _check("loopvq_codebook_update", _lib.loopvq_codebook_update(
+        ctypes.byref(desc), kind, _ptr(x), xd, n_tokens, stride_t, stride_n, stride_h, _ptr(idx_pool), tok_off,
+        pool_tokens, _ptr(cb_in), _ptr(cb_out), _ptr(counts_out) if counts_out is not None else None,
+        _ptr(workspace), _nbytes(workspace), _stream(stream)))
 
 
 def loopvq_decode_workspace_bytes(desc, layout) -> int:
