@@ -102,6 +102,12 @@ typedef struct {
  * only after it has).  Without the flag nothing is read before then.
  */
 #define LOOPVQ_LAYOUT_STATIC_INPUTS 0x1u
+/* The body lives in pages of the index pool listed by body_pages (see below)
+ * instead of at body_off. */
+#define LOOPVQ_LAYOUT_PAGED_BODY 0x2u
+/* The recent tokens live in a ring of win_ring slots per request (see below)
+ * instead of right after the sink tokens. */
+#define LOOPVQ_LAYOUT_RING_WINDOW 0x4u
 
 /*
  * Cache layout of one decode batch.  Request r has ctx_len[r] tokens, the
@@ -126,6 +132,28 @@ typedef struct {
   const int64_t* win_off;     /* device [batch] */
   int64_t body_pool_tokens;   /* capacity of each index pool stream, multiple of 32 */
   int64_t win_pool_tokens;    /* capacity of each window pool stream */
+  /* LOOPVQ_LAYOUT_PAGED_BODY (body_off is then ignored): body token p of
+   * request r sits at index-pool position
+   *   body_pages[r * max_body_pages + p / body_page_tokens] * body_page_tokens
+   *     + p % body_page_tokens.
+   * A page id outside [0, body_pool_tokens / body_page_tokens) sets
+   * LOOPVQ_FAULT_POOL_RANGE and that page is skipped. */
+  const int32_t* body_pages;  /* device [batch][max_body_pages], or NULL */
+  int32_t body_page_tokens;   /* a multiple of 32 (and of page) */
+  int32_t max_body_pages;     /* >= ceil(max body tokens / body_page_tokens) */
+  /* LOOPVQ_LAYOUT_RING_WINDOW: request r's window region starts at win_off[r]
+   * with n_sink sink slots, then a ring of win_ring slots; sink token i is at
+   * win_off[r] + i and recent token k (oldest first) at
+   *   win_off[r] + n_sink + (win_head[r] + k) % win_ring. */
+  const int32_t* win_head;    /* device [batch], or NULL */
+  int32_t win_ring;           /* >= n_recent + page - 1 */
+  int32_t reserved;           /* 0 */
+  /* The current token's key and value at this loop step, device bf16
+   * [batch][n_heads_kv][head_dim], or NULL.  When set, the decode uses them
+   * for the current token (the last window token) and also stores them in
+   * its window slot -- the pages' "write in bf16" fused into attention. */
+  const void* new_k;
+  const void* new_v;
 } loopvq_cache_layout;
 
 /* ------------------------------------------------------------------ info */

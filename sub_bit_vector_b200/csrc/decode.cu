@@ -86,7 +86,32 @@ struct DecodeParams {
   int split_len;   // body tokens per split (multiple of 32, <= kSplitCap)
   int max_splits;  // grid.x
   int static_inputs;  // layout arrays, index pools and codebooks are not being written by earlier kernels
+  // paged body: body token p at pool position body_pages[r][p / bpt] * bpt + p % bpt
+  int paged;
+  const int32_t* body_pages;
+  int body_page_tokens, max_body_pages;
+  // ring window: recent token k at win_off + n_sink + (win_head + k) % win_ring
+  int ring;
+  const int32_t* win_head;
+  int win_ring;
+  // the current token's K and V of this step ([batch][H][D] bf16), or null
+  const __nv_bfloat16* new_k;
+  const __nv_bfloat16* new_v;
 };
+
+// Window-pool row of window token i (sink tokens first, then the recent ones
+// oldest first).
+__device__ __forceinline__ int64_t win_row(const DecodeParams& p, int64_t win_off, int sink, int whead, int i) {
+  if (!p.ring || i < sink) return win_off + i;
+  return win_off + p.n_sink + (whead + (i - sink)) % p.win_ring;
+}
+// Rows i .. i+len-1 that are contiguous in the pool, starting at window token i.
+__device__ __forceinline__ int win_run(const DecodeParams& p, int sink, int whead, int i, int end) {
+  if (!p.ring) return end - i;
+  if (i < sink) return min(end, sink) - i;
+  const int slot = (whead + (i - sink)) % p.win_ring;
+  return min(end - i, p.win_ring - slot);
+}
 
 // Programmatic dependent launch: the kernel is launched so that it may start
 // while the previous kernel in the stream finishes.  Everything that kernel
@@ -376,9 +401,15 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
   if (split >= n_splits) return;
   const bool is_window = has_win && split == n_body_splits;  // partial row n_body_splits
   const int bsplit = split;
+  const int whead = (is_window && p.ring) ? __ldg(p.win_head + r) : 0;
   if (is_window) {
-    if (win_off < 0 || win_off + n_win > p.win_pool_tokens) bad = true;
-  } else {
+    if (p.ring) {
+      if (win_off < 0 || win_off + p.n_sink + p.win_ring > p.win_pool_tokens || whead < 0 || whead >= p.win_ring)
+        bad = true;
+    } else if (win_off < 0 || win_off + n_win > p.win_pool_tokens) {
+      bad = true;
+    }
+  } else if (!p.paged) {
     if (body_off < 0 || (body_off & 31) || body_off + cs.body > p.body_pool_tokens) bad = true;
   }
   if (bad && tid == 0) set_fault(p.status, LOOPVQ_FAULT_POOL_RANGE);
@@ -434,47 +465,91 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
   __syncthreads();
 
   // ======================= producer warp ===================================
+  // All 32 lanes walk the chunks (they hold a window of the page table for
+  // the paged body); lane 0 issues the barrier operations and the copies.
   if (warp == kNW) {
-    if (lane == 0) {
-      const uint8_t* vslice = reinterpret_cast<const uint8_t*>(p.cbV_slice) + (size_t)h * p.C * D * sizeof(CBT);
-      const uint32_t vslice_bytes = (uint32_t)(p.C * D * sizeof(CBT));
-      if (!is_window && n_tok > 0) prefetch_l2(vslice, vslice_bytes);  // the epilogue's codebook slice
-      if (is_window && p.static_inputs) griddep_wait();  // window rows may come from the previous kernel
-      const int n_slice = (is_window || n_tok == 0) ? 0 : (int)((vslice_bytes + kStageBytes - 1) / kStageBytes);
-      for (int k = 0; k < n_chunks + n_slice; ++k) {
-        const int s = k % kStages;
-        if (k == kPreWaitChunks && p.static_inputs && !is_window) griddep_wait();
-        if (k >= kStages) {
-          if (!mbar_wait_bounded(smem_u32(empty_bar + s), ((k / kStages) - 1) & 1)) {
-            set_fault(p.status, LOOPVQ_FAULT_TIMEOUT);
-            break;
-          }
+    const bool leader = lane == 0;
+    const uint8_t* vslice = reinterpret_cast<const uint8_t*>(p.cbV_slice) + (size_t)h * p.C * D * sizeof(CBT);
+    const uint32_t vslice_bytes = (uint32_t)(p.C * D * sizeof(CBT));
+    if (leader && !is_window && n_tok > 0) prefetch_l2(vslice, vslice_bytes);  // the epilogue's codebook slice
+    if (is_window && p.static_inputs) griddep_wait();  // window rows may come from the previous kernel
+    const int n_slice = (is_window || n_tok == 0) ? 0 : (int)((vslice_bytes + kStageBytes - 1) / kStageBytes);
+    const int32_t* pages = p.paged ? p.body_pages + (size_t)r * p.max_body_pages : nullptr;
+    const int64_t n_phys = p.paged ? p.body_pool_tokens / p.body_page_tokens : 0;
+    int pbase = -1 << 30, pcache = -1;  // page ids pbase + lane
+    for (int k = 0; k < n_chunks + n_slice; ++k) {
+      const int s = k % kStages;
+      if (k == kPreWaitChunks && p.static_inputs && !is_window) griddep_wait();
+      if (k >= kStages) {
+        int ok = 1;
+        if (leader) ok = mbar_wait_bounded(smem_u32(empty_bar + s), ((k / kStages) - 1) & 1) ? 1 : 0;
+        if (!__shfl_sync(0xffffffffu, ok, 0)) {
+          if (leader) set_fault(p.status, LOOPVQ_FAULT_TIMEOUT);
+          break;
         }
-        const uint32_t dst = stage_a[s];
-        const uint32_t fb = smem_u32(full_bar + s);
-        if (k >= n_chunks) {  // a piece of the value codebook slice, for the epilogue
-          const uint32_t off = (uint32_t)(k - n_chunks) * kStageBytes;
-          const uint32_t bytes = min((uint32_t)kStageBytes, vslice_bytes - off);
+      }
+      const uint32_t dst = stage_a[s];
+      const uint32_t fb = smem_u32(full_bar + s);
+      if (k >= n_chunks) {  // a piece of the value codebook slice, for the epilogue
+        const uint32_t off = (uint32_t)(k - n_chunks) * kStageBytes;
+        const uint32_t bytes = min((uint32_t)kStageBytes, vslice_bytes - off);
+        if (leader) {
           mbar_arrive_expect_tx(fb, bytes);
           bulk_g2s(dst, vslice + off, bytes, fb);
-        } else if (is_window) {
-          const bool vpass = k >= n_chunks_half;
-          const int t0 = (vpass ? k - n_chunks_half : k) * kRowsPerChunk;
-          const int nt = min(kRowsPerChunk, n_tok - t0);
-          const uint32_t bytes = (uint32_t)nt * D * 2;
-          const size_t row0 = ((size_t)h * p.win_pool_tokens + win_off + t0) * D;
-          mbar_arrive_expect_tx(fb, bytes);
-          bulk_g2s(dst, (vpass ? p.winV : p.winK) + row0, bytes, fb);
+        }
+      } else if (is_window) {
+        const bool vpass = k >= n_chunks_half;
+        const int t0 = (vpass ? k - n_chunks_half : k) * kRowsPerChunk;
+        const int t1 = min(n_tok, t0 + kRowsPerChunk);
+        const __nv_bfloat16* base = (vpass ? p.winV : p.winK) + (size_t)h * p.win_pool_tokens * D;
+        if (leader) {
+          mbar_arrive_expect_tx(fb, (uint32_t)(t1 - t0) * D * 2);
+          for (int i = t0; i < t1;) {  // contiguous runs of rows (a ring wraps once at most)
+            const int len = win_run(p, cs.sink, whead, i, t1);
+            bulk_g2s(dst + (uint32_t)(i - t0) * D * 2, base + win_row(p, win_off, cs.sink, whead, i) * D,
+                     (uint32_t)len * D * 2, fb);
+            i += len;
+          }
+        }
+      } else {
+        const bool vpass = k >= n_chunks_half;
+        const int c = vpass ? k - n_chunks_half : k;
+        const int tl0 = c * kTilesPerChunk;
+        const int nt = min(kTilesPerChunk, n_tiles - tl0);
+        const uint8_t* stream = (vpass ? p.idxV : p.idxK) + (int64_t)h * (p.body_pool_tokens >> 5) * (32 * J);
+        if (!p.paged) {
+          if (leader) {
+            const int64_t tile = ((body_off + tok0) >> 5) + tl0;
+            mbar_arrive_expect_tx(fb, (uint32_t)nt * 32 * J);
+            bulk_g2s(dst, stream + tile * (32 * J), (uint32_t)nt * 32 * J, fb);
+          }
         } else {
-          const bool vpass = k >= n_chunks_half;
-          const int c = vpass ? k - n_chunks_half : k;
-          const int tl0 = c * kTilesPerChunk;
-          const int nt = min(kTilesPerChunk, n_tiles - tl0);
-          const uint32_t bytes = (uint32_t)nt * 32 * J;
-          const int64_t tile = ((body_off + tok0) >> 5) + tl0;
-          const uint8_t* src = (vpass ? p.idxV : p.idxK) + ((int64_t)h * (p.body_pool_tokens >> 5) + tile) * (32 * J);
-          mbar_arrive_expect_tx(fb, bytes);
-          bulk_g2s(dst, src, bytes, fb);
+          // logical body tokens [a, e) split at page boundaries; invalid pages
+          // are reported and skipped (their bytes are not expected)
+          const int a = tok0 + tl0 * 32, e = a + nt * 32;
+          const int bpt = p.body_page_tokens;
+          uint32_t valid = 0;
+          for (int pass = 0; pass < 2; ++pass) {
+            if (pass == 1 && leader) mbar_arrive_expect_tx(fb, valid);
+            for (int t = a; t < e;) {
+              const int pi = t / bpt;
+              const int len = min(e - t, bpt - t % bpt);
+              if (pi < pbase || pi >= pbase + 32) {  // warp-uniform
+                pbase = pi;
+                pcache = pbase + lane < p.max_body_pages ? __ldg(pages + pbase + lane) : -1;
+              }
+              const int phys = __shfl_sync(0xffffffffu, pcache, pi - pbase);
+              const bool ok = pi < p.max_body_pages && phys >= 0 && phys < n_phys;
+              if (pass == 0) {
+                if (ok) valid += (uint32_t)len * J;
+                else if (leader) set_fault(p.status, LOOPVQ_FAULT_POOL_RANGE);
+              } else if (ok && leader) {
+                const int64_t pos = (int64_t)phys * bpt + t % bpt;  // a multiple of 32
+                bulk_g2s(dst + (uint32_t)(t - a) * J, stream + (pos >> 5) * (32 * J), (uint32_t)len * J, fb);
+              }
+              t += len;
+            }
+          }
         }
       }
     }
@@ -497,12 +572,41 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
       qv[i] = load_q(p.q, p.q_bf16, unit * D + lane * CPL + i) * p.scale_log2;
       ov[i] = 0.f;
     }
+    // The current token is the last window token.  With new_k/new_v given,
+    // its row in the stage is replaced by them (the pool row may not hold it
+    // yet), and one CTA per KV head also stores them into the window pool.
+    const int i_cur = n_tok - 1;
+    const bool has_new = p.new_k != nullptr && n_tok > 0;
+    if (has_new && hq % group == 0 && warp == 0) {
+      const int64_t row = win_row(p, win_off, cs.sink, whead, i_cur);
+      const size_t src = ((size_t)r * p.H + h) * D + lane * CPL;
+      const size_t dstp = ((size_t)h * p.win_pool_tokens + row) * D + lane * CPL;
+      __nv_bfloat16* wk = const_cast<__nv_bfloat16*>(p.winK);
+      __nv_bfloat16* wv = const_cast<__nv_bfloat16*>(p.winV);
+#pragma unroll
+      for (int i = 0; i < CPL; ++i) {
+        wk[dstp + i] = p.new_k[src + i];
+        wv[dstp + i] = p.new_v[src + i];
+      }
+    }
+    // overwrite row i_cur - t0 of a stage that holds window tokens from t0
+    auto patch_row = [&](uint8_t* st, int t0, const __nv_bfloat16* nv) {
+      if (warp == 0) {
+        const __nv_bfloat16* src = nv + ((size_t)r * p.H + h) * D + lane * CPL;
+        __nv_bfloat16* d = reinterpret_cast<__nv_bfloat16*>(st + (size_t)(i_cur - t0) * D * 2) + lane * CPL;
+#pragma unroll
+        for (int i = 0; i < CPL; ++i) d[i] = src[i];
+        fence_proxy_async();  // the stage is refilled by TMA later
+      }
+      consumer_sync();
+    };
     float mx = -INFINITY;
     for (int k = 0; k < n_chunks_half; ++k) {
       const int s = k % kStages;
       if (!mbar_wait_bounded(smem_u32(full_bar + s), (k / kStages) & 1)) set_fault(p.status, LOOPVQ_FAULT_TIMEOUT);
       const uint8_t* st = stage_ptr(s);
       const int nt = min(kRowsPerChunk, n_tok - k * kRowsPerChunk);
+      if (has_new && i_cur / kRowsPerChunk == k) patch_row(stage_ptr(s), k * kRowsPerChunk, p.new_k);
       for (int b0 = warp; b0 < nt; b0 += 4 * kNW) {
         float dot[4];
 #pragma unroll
@@ -549,6 +653,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
       const uint8_t* st = stage_ptr(s);
       const int kv = k - n_chunks_half;
       const int nt = min(kRowsPerChunk, n_tok - kv * kRowsPerChunk);
+      if (has_new && i_cur / kRowsPerChunk == kv) patch_row(stage_ptr(s), kv * kRowsPerChunk, p.new_v);
       for (int tkn = warp; tkn < nt; tkn += kNW) {
         const float pw = exp2f(sc[kv * kRowsPerChunk + tkn] - m);
         const uint8_t* vr = st + (size_t)tkn * D * 2 + lane * CPL * 2;
@@ -855,9 +960,36 @@ static WsLayout decode_ws(const Geo& g, const loopvq_cache_layout* L) {
 static loopvq_status check_layout(const loopvq_cache_layout* L) {
   if (!L || L->batch < 1 || L->n_sink < 0 || L->n_recent < 0 || L->page < 1 || L->max_ctx_len < 0)
     return LOOPVQ_ERR_INVALID_ARG;
-  if (!L->ctx_len || !L->body_off || !L->win_off) return LOOPVQ_ERR_INVALID_ARG;
+  const bool paged = L->flags & LOOPVQ_LAYOUT_PAGED_BODY, ring = L->flags & LOOPVQ_LAYOUT_RING_WINDOW;
+  if (L->flags & ~(LOOPVQ_LAYOUT_STATIC_INPUTS | LOOPVQ_LAYOUT_PAGED_BODY | LOOPVQ_LAYOUT_RING_WINDOW))
+    return LOOPVQ_ERR_INVALID_ARG;
+  if (!L->ctx_len || !L->win_off || (!paged && !L->body_off)) return LOOPVQ_ERR_INVALID_ARG;
   if (L->body_pool_tokens < 0 || (L->body_pool_tokens & 31) || L->win_pool_tokens < 0) return LOOPVQ_ERR_INVALID_ARG;
+  if (paged) {
+    if (!L->body_pages || L->body_page_tokens < 32 || (L->body_page_tokens & 31) ||
+        L->body_page_tokens % L->page || L->max_body_pages < 1)
+      return LOOPVQ_ERR_INVALID_ARG;
+    const int64_t body = ctx_split(L->max_ctx_len, L->n_sink, L->n_recent, L->page).body;
+    if ((int64_t)L->max_body_pages * L->body_page_tokens < body) return LOOPVQ_ERR_INVALID_ARG;
+  }
+  if (ring && (!L->win_head || L->win_ring < 1 || L->win_ring < L->n_recent + L->page - 1))
+    return LOOPVQ_ERR_INVALID_ARG;
+  if ((L->new_k == nullptr) != (L->new_v == nullptr)) return LOOPVQ_ERR_INVALID_ARG;
+  if (((uintptr_t)L->new_k & 3) || ((uintptr_t)L->new_v & 3)) return LOOPVQ_ERR_INVALID_ARG;
   return LOOPVQ_OK;
+}
+
+// Layout fields of the kernel parameters shared by both entry points.
+static void fill_layout_params(DecodeParams& p, const loopvq_cache_layout* L) {
+  p.paged = (L->flags & LOOPVQ_LAYOUT_PAGED_BODY) ? 1 : 0;
+  p.body_pages = L->body_pages;
+  p.body_page_tokens = p.paged ? L->body_page_tokens : 32;
+  p.max_body_pages = L->max_body_pages;
+  p.ring = (L->flags & LOOPVQ_LAYOUT_RING_WINDOW) ? 1 : 0;
+  p.win_head = L->win_head;
+  p.win_ring = p.ring ? L->win_ring : 1;
+  p.new_k = (const __nv_bfloat16*)L->new_k;
+  p.new_v = (const __nv_bfloat16*)L->new_v;
 }
 
 }  // namespace loopvq
@@ -932,6 +1064,7 @@ extern "C" loopvq_status loopvq_decode_attn(const loopvq_codebook_desc* desc, co
   p.max_splits = pl.max_splits;
 
   p.static_inputs = (layout->flags & LOOPVQ_LAYOUT_STATIC_INPUTS) ? 1 : 0;
+  fill_layout_params(p, layout);
 
   dim3 grid(g.Hq, pl.max_splits, layout->batch);
   cudaStream_t s = (cudaStream_t)stream;
@@ -1068,6 +1201,7 @@ extern "C" loopvq_status loopvq_decode_attn_noalloc(const loopvq_codebook_desc* 
   p.max_splits = pl.max_splits;
 
   p.static_inputs = (layout->flags & LOOPVQ_LAYOUT_STATIC_INPUTS) ? 1 : 0;
+  fill_layout_params(p, layout);
 
   dim3 grid(g.Hq, pl.max_splits, layout->batch);
 #define LOOPVQ_LAUNCH(JJ, DD, CBT)                                                                    \

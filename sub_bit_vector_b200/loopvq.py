@@ -33,6 +33,8 @@ LOOPVQ_FAULT_POOL_RANGE = 0x4
 LOOPVQ_FAULT_TIMEOUT = 0x8
 
 LOOPVQ_LAYOUT_STATIC_INPUTS = 0x1
+LOOPVQ_LAYOUT_PAGED_BODY = 0x2
+LOOPVQ_LAYOUT_RING_WINDOW = 0x4
 
 EXPORTED = [
     "loopvq_version", "loopvq_status_string", "loopvq_validate_desc", "loopvq_ctx_split",
@@ -62,7 +64,10 @@ class loopvq_cache_layout(ctypes.Structure):
     _fields_ = [("batch", ctypes.c_int32), ("n_sink", ctypes.c_int32), ("n_recent", ctypes.c_int32),
                 ("page", ctypes.c_int32), ("max_ctx_len", ctypes.c_int32), ("flags", ctypes.c_uint32),
                 ("ctx_len", ctypes.c_void_p), ("body_off", ctypes.c_void_p), ("win_off", ctypes.c_void_p),
-                ("body_pool_tokens", ctypes.c_int64), ("win_pool_tokens", ctypes.c_int64)]
+                ("body_pool_tokens", ctypes.c_int64), ("win_pool_tokens", ctypes.c_int64),
+                ("body_pages", ctypes.c_void_p), ("body_page_tokens", ctypes.c_int32),
+                ("max_body_pages", ctypes.c_int32), ("win_head", ctypes.c_void_p), ("win_ring", ctypes.c_int32),
+                ("reserved", ctypes.c_int32), ("new_k", ctypes.c_void_p), ("new_v", ctypes.c_void_p)]
 
 
 def _load() -> ctypes.CDLL:
@@ -159,9 +164,12 @@ def make_desc(n_loop, tc, n_heads_kv, head_dim, group_elems, n_codes=256, n_head
 
 
 def make_layout(batch, n_sink, n_recent, page, max_ctx_len, ctx_len, body_off, win_off,
-                body_pool_tokens, win_pool_tokens, flags=0) -> loopvq_cache_layout:
+                body_pool_tokens, win_pool_tokens, flags=0, body_pages=None, body_page_tokens=0,
+                max_body_pages=0, win_head=None, win_ring=0, new_k=None, new_v=None) -> loopvq_cache_layout:
     return loopvq_cache_layout(batch, n_sink, n_recent, page, max_ctx_len, flags, _ptr(ctx_len), _ptr(body_off),
-                               _ptr(win_off), body_pool_tokens, win_pool_tokens)
+                               _ptr(win_off), body_pool_tokens, win_pool_tokens, _ptr(body_pages),
+                               body_page_tokens, max_body_pages, _ptr(win_head), win_ring, 0, _ptr(new_k),
+                               _ptr(new_v))
 
 
 # ------------------------------------------------------------------ entry points
