@@ -406,30 +406,42 @@ def run_gpu(args):
                 "frac_of_8TBps_spec": achieved / 8000.0}
 
     # ---- end to end through the public API with host buffers: every step
-    # copies the 4 loop steps' queries and the new token's bf16 K/V (written
-    # into the recent window) from pinned host memory, runs the 4 decode
-    # calls (and the page encode every 8th step) and reads the fp32 outputs
-    # back into pinned host memory.
+    # copies the 4 loop steps' queries and the new token's bf16 K and V from
+    # pinned host memory in one transfer, runs the 4 decode calls -- each
+    # writes the new token's K/V of its step into the recent window itself
+    # (the layout's new_k/new_v) -- plus the page encode every 8th step, and
+    # reads the 4 fp32 outputs back into pinned host memory.
     e2e_steps = min(args.steps, 2000)
-    q_host = torch.randn((T, 1, H, D), generator=torch.Generator().manual_seed(5)).to(torch.bfloat16).pin_memory()
-    kv_host = torch.randn((2, T, H, D), generator=torch.Generator().manual_seed(6)).to(torch.bfloat16).pin_memory()
+    n_q = T * H * D
+    in_host = torch.randn(3 * n_q, generator=torch.Generator().manual_seed(5)).to(torch.bfloat16).pin_memory()
     out_host = torch.empty((T, 1, H, D), dtype=torch.float32).pin_memory()
-    kv_dev = torch.empty((2, T, H, D), dtype=torch.bfloat16, device=device)
-    h2d = q_host.numel() * 2 + kv_host.numel() * 2
+    in_dev = torch.empty(3 * n_q, dtype=torch.bfloat16, device=device)
+    q_dev = in_dev[:n_q].view(T, 1, H, D)
+    k_dev = in_dev[n_q:2 * n_q].view(T, 1, H, D)
+    v_dev = in_dev[2 * n_q:].view(T, 1, H, D)
+    out_dev = torch.empty((T, 1, H, D), dtype=torch.float32, device=device)
+    lse_dev = torch.empty((T, 1, H), dtype=torch.float32, device=device)
+    h2d = in_host.numel() * 2
     d2h = out_host.numel() * 4
-    pos = N_SINK + N_RECENT - 1          # slot of the newest token in the window pool
+    calls = []
+    for c in layers:
+        per = []
+        for t in range(T):
+            lay = L.make_layout(1, N_SINK, N_RECENT, PAGE, c.max_ctx_len, c.ctx_dev, c.body_off_dev, c.win_off_dev,
+                                c.body_pool_tokens, c.win_pool_tokens, L.LOOPVQ_LAYOUT_STATIC_INPUTS,
+                                new_k=k_dev[t], new_v=v_dev[t])
+            per.append(L.prepare_decode_attn(c.desc, c.cbK, c.cbV, lay, c.idxK, c.idxV, c.winK, c.winV, q_dev[t], t,
+                                             D ** -0.5, out_dev[t], lse_dev[t], c.workspace, stream))
+        calls.append(per)
     with torch.cuda.stream(stream):
         def e2e_step(i):
-            c = layers[i % N_LAYERS]
-            kv_dev.copy_(kv_host, non_blocking=True)
-            c.winK[:, :, pos].copy_(kv_dev[0])
-            c.winV[:, :, pos].copy_(kv_dev[1])
+            li = i % N_LAYERS
+            in_dev.copy_(in_host, non_blocking=True)
             for t in range(T):
-                c.q.copy_(q_host[t], non_blocking=True)
-                c.decode(t, stream=stream)
-                out_host[t].copy_(c.out, non_blocking=True)
+                calls[li][t]()
             if i % PAGE == PAGE - 1:
-                encode_page(c, stream)
+                encode_page(layers[li], stream)
+            out_host.copy_(out_dev, non_blocking=True)
             stream.synchronize()
         for i in range(min(args.warmup, 50)):
             e2e_step(i)
@@ -446,8 +458,9 @@ def run_gpu(args):
     e2e_ms = reduce_over_ranks([s0.elapsed_time(s1)], world, device)[0]
     e2e = {"value": aggregate_value(world, e2e_steps, tokens_per_step, e2e_ms), "unit": UNIT,
            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": e2e_steps,
-           "path": "pinned host q + new-token K/V -> device, 4 loopvq_decode_attn calls (+ page encode every "
-                   "8th step), fp32 outputs -> pinned host, stream sync per step"}
+           "path": "pinned host queries + new-token K/V -> device in one copy, 4 loopvq_decode_attn calls that "
+                   "also write the new token into the window (+ page encode every 8th step), fp32 outputs -> "
+                   "pinned host, stream sync per step"}
 
     dense = dense_comparator(device) if not args.no_extras else None
     launches = args.steps * T + 2 * n_enc_steps

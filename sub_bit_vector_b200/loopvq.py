@@ -266,6 +266,26 @@ def loopvq_decode_attn(desc, cbK_packed, cbV_packed, layout, idxK_pool, idxV_poo
         _ptr(out), _dtype_code(out), _ptr(lse_out), _ptr(workspace), wb, _stream(stream)))
 
 
+def prepare_decode_attn(desc, cbK_packed, cbV_packed, layout, idxK_pool, idxV_pool, winK, winV, q, loop_step,
+                        softmax_scale, out, lse_out, workspace, stream=None):
+    """loopvq_decode_attn with every argument marshalled once: returns a
+    zero-argument callable that issues the call (for per-token loops where
+    the buffers stay put and the Python-side argument conversion would cost
+    more than the launch).  The tensors must stay alive and in place."""
+    fn = _lib.loopvq_decode_attn
+    args = (ctypes.byref(desc), _ptr(cbK_packed), _ptr(cbV_packed), ctypes.byref(layout), _ptr(idxK_pool),
+            _ptr(idxV_pool), _ptr(winK), _ptr(winV), _ptr(q), _dtype_code(q), loop_step, softmax_scale, _ptr(out),
+            _dtype_code(out), _ptr(lse_out), _ptr(workspace), _nbytes(workspace), _stream(stream))
+    keep = (desc, layout)
+
+    def call():
+        st = fn(*args)
+        if st != LOOPVQ_OK:
+            raise LoopVQError("loopvq_decode_attn", st)
+    call._keep = keep
+    return call
+
+
 def loopvq_decode_attn_noalloc(desc, cbK_packed, cbV_packed, layout, idxK_pool, idxV_pool, winK, winV, q,
                                loop_step, softmax_scale, out, lse_out, fault_bits=None, stream=None) -> None:
     """Same as loopvq_decode_attn but with no workspace: for callers that
