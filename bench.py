@@ -463,7 +463,7 @@ def run_gpu(args):
                    "pinned host, stream sync per step"}
 
     dense = dense_comparator(device) if not args.no_extras else None
-    launches = args.steps * T + 2 * n_enc_steps
+    launches = args.steps * T * 2 + 2 * n_enc_steps   # decode + merge kernel per loop step; K and V page encodes
     if rank == 0:
         line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,

@@ -21,8 +21,8 @@
 //                histogram hist[j][idxV[n][j]] with shared-memory integer
 //                atomics (same rotation: conflict free).
 //     epilogue   -- o[jW+w] = 2^-S sum_c hist[j][c] B^V_t[c][j][w].
-//   The last CTA of a (request, head) merges the splits' (m, l, o) by
-//   log-sum-exp (atomic ticket, no waiting).
+//   Every split writes its (m, l, o); a small merge kernel, launched right
+//   after as a programmatic dependent, combines them by log-sum-exp.
 //
 // Fixed-point bound: a split holds n <= kSplitCap < 2^12 tokens and S is
 // chosen so that n * 2^S < 2^32, so no bin or sum can overflow.
@@ -124,9 +124,6 @@ __device__ __forceinline__ void griddep_launch_dependents() { asm volatile("grid
 __device__ __forceinline__ void consumer_sync() {
   asm volatile("bar.sync 1, %0;" ::"n"(kNW * 32) : "memory");
 }
-struct ConsumerSync {
-  __device__ __forceinline__ void operator()() const { consumer_sync(); }
-};
 
 __device__ __forceinline__ float lds_f32(uint32_t a) {
   float v;
@@ -275,69 +272,6 @@ __device__ __forceinline__ float load_q(const void* q, int q_bf16, size_t i) {
                 : reinterpret_cast<const float*>(q)[i];
 }
 
-// Last-split merge with one global round trip: every split's (o, m, l) row is
-// staged in shared memory (`sm`, `cap` floats), then combined there.  Falls
-// back to the two-phase combine when the rows do not fit.
-__device__ __forceinline__ void combine_staged(const float* part, int n_splits, int D, void* out, int out_bf16,
-                                               float* lse, float* sm, int cap, int tid, int nthr) {
-  const int row = D + 4;
-  const int n4 = n_splits * row / 4;  // rows are 16-byte multiples
-  if (n_splits * row > cap || n4 > 4 * nthr || n_splits > 64) {
-    combine_splits(part, n_splits, D, out, out_bf16, lse, sm, tid, nthr, ConsumerSync{});
-    return;
-  }
-  // every partial in flight at once: one round trip to L2
-  const float4* src = reinterpret_cast<const float4*>(part);
-  float4 v[4];
-#pragma unroll
-  for (int u = 0; u < 4; ++u) {
-    const int i = tid + u * nthr;
-    if (i < n4) v[u] = __ldcg(src + i);
-  }
-#pragma unroll
-  for (int u = 0; u < 4; ++u) {
-    const int i = tid + u * nthr;
-    if (i < n4) reinterpret_cast<float4*>(sm)[i] = v[u];
-  }
-  consumer_sync();
-  // Each warp that writes outputs derives the merge weights 2^(m_s - M) / L
-  // itself (lane s holds splits s and s + 32), so no second barrier.
-  if (tid < D) {
-    const int lane = tid & 31;
-    float ms[2], ls[2];
-#pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      const int s = lane + 32 * u;
-      ms[u] = s < n_splits ? sm[s * row + D] : -INFINITY;
-      ls[u] = s < n_splits ? sm[s * row + D + 1] : 0.f;
-    }
-    float M = fmaxf(ms[0], ms[1]);
-#pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-    float e[2], L = 0.f;
-#pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      e[u] = ms[u] == -INFINITY ? 0.f : exp2f(ms[u] - M);
-      L = fmaf(ls[u], e[u], L);
-    }
-#pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
-    const bool ok = M != -INFINITY && L > 0.f;
-    const float inv = ok ? __frcp_rn(L) : 0.f;
-    const float w0 = e[0] * inv, w1 = e[1] * inv;
-    float o4[4] = {0.f, 0.f, 0.f, 0.f};
-    const int n0 = n_splits < 32 ? n_splits : 32;
-    for (int s = 0; s < n0; ++s) o4[s & 3] = fmaf(sm[s * row + tid], __shfl_sync(0xffffffffu, w0, s), o4[s & 3]);
-    for (int s = 32; s < n_splits; ++s) o4[s & 3] = fmaf(sm[s * row + tid], __shfl_sync(0xffffffffu, w1, s - 32), o4[s & 3]);
-    const float r = (o4[0] + o4[1]) + (o4[2] + o4[3]);
-    if (out_bf16)
-      ((__nv_bfloat16*)out)[tid] = __float2bfloat16_rn(r);
-    else
-      ((float*)out)[tid] = r;
-    if (lse && tid == 0) *lse = ok ? (M + log2f(L)) * 0.6931471805599453f : -INFINITY;
-  }
-}
-
 template <int J, int D, typename CBT>
 __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams p) {
   extern __shared__ __align__(1024) uint8_t dyn[];
@@ -387,17 +321,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
   const int has_win = n_win > 0 ? 1 : 0;
   const int n_body_splits = (cs.body + p.split_len - 1) / p.split_len;
   const int n_splits = has_win + n_body_splits;
-  if (ctx == 0) {  // empty context: zero output, lse -inf
-    if (split == 0) {
-      griddep_wait();
-      for (int d = tid; d < D; d += blockDim.x) {
-        if (p.out_bf16) reinterpret_cast<__nv_bfloat16*>(p.out)[unit * D + d] = __float2bfloat16_rn(0.f);
-        else reinterpret_cast<float*>(p.out)[unit * D + d] = 0.f;
-      }
-      if (p.lse && tid == 0) p.lse[unit] = -INFINITY;
-    }
-    return;
-  }
+  if (ctx == 0) return;  // empty context: the merge kernel writes a zero output
   if (split >= n_splits) return;
   const bool is_window = has_win && split == n_body_splits;  // partial row n_body_splits
   const int bsplit = split;
@@ -445,7 +369,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
   uint64_t* const full_bar = reinterpret_cast<uint64_t*>(misc);
   uint64_t* const empty_bar = full_bar + kStages;
   float* const red = reinterpret_cast<float*>(misc + 256);          // [kNW * 2]
-  int* const flag = reinterpret_cast<int*>(misc + 512);
 
   // chunks: window -> K rows then V rows, kRowsPerChunk tokens each;
   //         body   -> K tiles then V tiles, kTilesPerChunk each.
@@ -885,35 +808,89 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
     }
   }
 
-  // ---- split ticket and combine -------------------------------------------
-  consumer_sync();
-  if (ctid == 0) {
-    // release: this CTA's partial (ordered before by the barrier) before the
-    // ticket; acquire: the other splits' partials after theirs
-    uint32_t t;
-    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(t) : "l"(p.tickets + unit) : "memory");
-    *flag = t == (uint32_t)(n_splits - 1);
+  // the merge kernel, launched right after as a dependent, combines the splits
+}
+
+// Merge of the splits of every (request, query head): one CTA per unit,
+// launched as a programmatic dependent of the decode kernel (it starts while
+// the decode runs and waits for its completion before reading the
+// partials).  Partials are staged 32 splits at a time, every load of a stage
+// in flight together; the log-sum-exp merge runs online across stages.
+constexpr int kMergeThreads = 256;
+constexpr int kMergeChunk = 32;
+
+template <int D>
+__global__ void __launch_bounds__(kMergeThreads) merge_kernel(const DecodeParams p) {
+  __shared__ __align__(16) float sm[kMergeChunk * (D + 4)];
+  griddep_launch_dependents();
+  const int tid = threadIdx.x, lane = tid & 31;
+  const int hq = blockIdx.x, r = blockIdx.y;
+  const size_t unit = (size_t)r * p.Hq + hq;
+  int ctx = __ldg(p.ctx_len + r);
+  if (ctx < 0 || ctx > p.max_ctx) ctx = 0;  // reported by the decode kernel
+  const CtxSplit cs = ctx_split(ctx, p.n_sink, p.n_recent, p.page);
+  const int n_win = cs.sink + cs.recent;
+  const int n_splits = ctx == 0 ? 0 : (n_win > 0 ? 1 : 0) + (cs.body + p.split_len - 1) / p.split_len;
+  griddep_wait();
+  const float* part = p.partials + unit * p.max_splits * (size_t)(D + 4);
+  constexpr int kPer = (kMergeChunk * (D + 4) / 4 + kMergeThreads - 1) / kMergeThreads;
+  float M = -INFINITY, Ls = 0.f, o = 0.f;  // running merge; thread d < D holds o[d]
+  for (int c0 = 0; c0 < n_splits; c0 += kMergeChunk) {
+    const int nc = min(kMergeChunk, n_splits - c0);
+    const int n4 = nc * (D + 4) / 4;
+    const float4* src = reinterpret_cast<const float4*>(part + (size_t)c0 * (D + 4));
+    float4 v[kPer];
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+      const int i = tid + u * kMergeThreads;
+      if (i < n4) v[u] = __ldcg(src + i);
+    }
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+      const int i = tid + u * kMergeThreads;
+      if (i < n4) reinterpret_cast<float4*>(sm)[i] = v[u];
+    }
+    __syncthreads();
+    if (tid < D) {
+      const float ms = lane < nc ? sm[lane * (D + 4) + D] : -INFINITY;
+      const float ls = lane < nc ? sm[lane * (D + 4) + D + 1] : 0.f;
+      float Mc = ms;
+#pragma unroll
+      for (int x = 16; x >= 1; x >>= 1) Mc = fmaxf(Mc, __shfl_xor_sync(0xffffffffu, Mc, x));
+      const float Mn = fmaxf(M, Mc);
+      const float e = ms == -INFINITY ? 0.f : exp2f(ms - Mn);
+      float Lc = ls * e;
+#pragma unroll
+      for (int x = 16; x >= 1; x >>= 1) Lc += __shfl_xor_sync(0xffffffffu, Lc, x);
+      const float keep = M == -INFINITY ? 0.f : exp2f(M - Mn);
+      float oc[4] = {0.f, 0.f, 0.f, 0.f};
+      for (int s = 0; s < nc; ++s) oc[s & 3] = fmaf(sm[s * (D + 4) + tid], __shfl_sync(0xffffffffu, e, s), oc[s & 3]);
+      o = fmaf(o, keep, (oc[0] + oc[1]) + (oc[2] + oc[3]));
+      Ls = fmaf(Ls, keep, Lc);
+      M = Mn;
+    }
+    __syncthreads();
   }
-  consumer_sync();
-  if (*flag) {
-    // the drained ring (stage 1) is the combine scratch
-    combine_staged(p.partials + unit * p.max_splits * (size_t)(D + 4), n_splits, D,
-                   p.out_bf16 ? (void*)(reinterpret_cast<__nv_bfloat16*>(p.out) + unit * D)
-                              : (void*)(reinterpret_cast<float*>(p.out) + unit * D),
-                   p.out_bf16, p.lse ? p.lse + unit : nullptr, reinterpret_cast<float*>(stage_ptr(1)),
-                   kStageBytes / 4, ctid, kNW * 32);
-    if (ctid == 0) atomicExch(p.tickets + unit, 0u);
+  if (tid < D) {
+    const bool ok = M != -INFINITY && Ls > 0.f;
+    const float res = ok ? o * __frcp_rn(Ls) : 0.f;
+    if (p.out_bf16)
+      reinterpret_cast<__nv_bfloat16*>(p.out)[unit * D + tid] = __float2bfloat16_rn(res);
+    else
+      reinterpret_cast<float*>(p.out)[unit * D + tid] = res;
+    if (p.lse && tid == 0) p.lse[unit] = ok ? (M + log2f(Ls)) * 0.6931471805599453f : -INFINITY;
   }
 }
 
 // Launches the decode kernel as a programmatic dependent of the previous
 // kernel in the stream (it may start while that kernel finishes; the kernel
 // waits for it before touching anything it may write).
-static cudaError_t launch_pdl(const void* fn, dim3 grid, cudaStream_t s, DecodeParams* p) {
+static cudaError_t launch_pdl(const void* fn, dim3 grid, cudaStream_t s, DecodeParams* p,
+                              unsigned threads = kThreads, size_t smem = kDynSmem) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
-  cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = kDynSmem;
+  cfg.blockDim = dim3(threads);
+  cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -1074,6 +1051,9 @@ extern "C" loopvq_status loopvq_decode_attn(const loopvq_codebook_desc* desc, co
     if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, kDynSmem) != cudaSuccess) \
       return LOOPVQ_ERR_CUDA;                                                                        \
     if (launch_pdl((const void*)kfn, grid, s, &p) != cudaSuccess) return LOOPVQ_ERR_CUDA;           \
+    if (launch_pdl((const void*)merge_kernel<DD>, dim3(g.Hq, layout->batch), s, &p, kMergeThreads, 0) != \
+        cudaSuccess)                                                                                 \
+      return LOOPVQ_ERR_CUDA;                                                                        \
   } while (0)
 #define LOOPVQ_LAUNCH_J(DD, CBT)                      \
   do {                                                \
@@ -1210,6 +1190,9 @@ extern "C" loopvq_status loopvq_decode_attn_noalloc(const loopvq_codebook_desc* 
     if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, kDynSmem) != cudaSuccess) \
       return LOOPVQ_ERR_CUDA;                                                                        \
     if (launch_pdl((const void*)kfn, grid, s, &p) != cudaSuccess) return LOOPVQ_ERR_CUDA;           \
+    if (launch_pdl((const void*)merge_kernel<DD>, dim3(g.Hq, layout->batch), s, &p, kMergeThreads, 0) != \
+        cudaSuccess)                                                                                 \
+      return LOOPVQ_ERR_CUDA;                                                                        \
   } while (0)
 #define LOOPVQ_LAUNCH_J(DD, CBT)                      \
   do {                                                \
