@@ -98,9 +98,27 @@ def cpu_baseline(budget_s: float = 15.0):
         t0 = time.perf_counter()
         pool.map(_oracle_task, tasks, chunksize=1)
         wall = time.perf_counter() - t0
+    per_task = sorted(per)[len(per) // 2]
     return {"value": n_tasks * CTX / wall, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "single_core_value": CTX / per_task,
             "sample": f"{n_tasks} (KV head, loop step) decode-attention problems of the 32K workload "
-                      f"(each 1 head x {CTX} tokens), spawn pool of {cores} processes, {wall:.1f} s wall"}
+                      f"(each 1 head x {CTX} tokens), spawn pool of {cores} processes, {wall:.1f} s wall; "
+                      f"single_core_value from the median warm-up task"}
+
+
+def encode_oracle_sample(x_host, cb_host):
+    """The oracle's nearest-codeword encode timed on a seeded 1/64 sample of
+    the prefill's tokens (all heads and slots), one process; sub-vectors/s."""
+    import numpy as np
+    import oracle as O
+    rng = np.random.Generator(np.random.PCG64(11))
+    toks = np.sort(rng.choice(x_host.shape[1], x_host.shape[1] // 64, replace=False))
+    xs = x_host[:, toks]
+    t0 = time.perf_counter()
+    O.encode(xs, cb_host, TC)
+    wall = time.perf_counter() - t0
+    n_sub = (T // TC) * H * (D // (G // TC)) * len(toks)
+    return n_sub / wall, f"{len(toks)} of {x_host.shape[1]} tokens (1/64, all heads and slots), 1 process"
 
 
 def run_reference(args):
@@ -297,6 +315,64 @@ def dense_comparator(device, reps=50):
             "kv_tokens_per_s": CTX / (us * 1e-6)}
 
 
+def sdpa_comparator(device, reps=50):
+    """torch's scaled_dot_product_attention on the bf16 cache of one loop step
+    (batch 1, 16 heads x 32768 tokens x 128, one query), for context."""
+    import torch
+    from sub_bit_vector_b200 import synth
+    n_buf = 2
+    ks = [synth.device_normal(1900 + i, (1, H, CTX, D), device=device) for i in range(n_buf)]
+    vs = [synth.device_normal(1950 + i, (1, H, CTX, D), device=device) for i in range(n_buf)]
+    q = synth.device_normal(1999, (1, H, 1, D), device=device)
+    f = torch.nn.functional.scaled_dot_product_attention
+    for i in range(4):
+        f(q, ks[i % n_buf], vs[i % n_buf])
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record()
+    for i in range(reps):
+        f(q, ks[i % n_buf], vs[i % n_buf])
+    e1.record()
+    torch.cuda.synchronize()
+    us = e0.elapsed_time(e1) * 1e3 / reps
+    return {"us_per_launch": us, "kv_tokens_per_s": CTX / (us * 1e-6), "what": "torch SDPA, bf16 K/V, 1 query"}
+
+
+def encode_measurement(device, with_oracle, reps=5):
+    """Loop-axis encode of a 32768-token prefill's keys [4][32768][16][128]
+    bf16 at 0.5 bit (tensor-core kernel); with_oracle adds the oracle's rate
+    on a 1/64 sample (host cores)."""
+    import torch
+    from sub_bit_vector_b200 import loopvq as L, synth
+    W = G // TC
+    J = D // W
+    x = synth.device_normal(2100, (T, CTX, H, D), device=device)
+    cb = synth.device_normal(2101, (T // TC, H, J, 256, TC, W), device=device)
+    desc = L.make_desc(T, TC, H, D, G)
+    packed = torch.zeros(L.loopvq_codebook_packed_bytes(desc), dtype=torch.uint8, device=device)
+    L.loopvq_codebook_pack(desc, cb, packed)
+    pool = torch.zeros(L.loopvq_index_pool_bytes(desc, CTX), dtype=torch.uint8, device=device)
+    args = (desc, packed, L.LOOPVQ_KEYS, x, CTX, CTX * H * D, H * D, D, pool, 0, CTX)
+    for _ in range(2):
+        L.loopvq_encode(*args)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record()
+    for _ in range(reps):
+        L.loopvq_encode(*args)
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / reps
+    n_sub = (T // TC) * H * J * CTX
+    res = {"kernel": "loopvq::encode_tc_kernel<16,32>", "ms_per_tensor": ms, "subvectors_per_s": n_sub / (ms * 1e-3),
+           "what": "keys [4][32768][16][128] bf16, Tc=4, G=16, 256 codes"}
+    if with_oracle:
+        rate, sample = encode_oracle_sample(x.float().cpu().numpy(), cb.float().cpu().numpy())
+        res["oracle_subvectors_per_s"] = rate
+        res["oracle_sample"] = sample
+    return res
+
+
 def reduce_over_ranks(values, world, device=None):
     """Max over ranks of per-rank device timings (ms); every rank takes the
     same collective step.  Returns the list of maxima."""
@@ -463,6 +539,9 @@ def run_gpu(args):
                    "pinned host, stream sync per step"}
 
     dense = dense_comparator(device) if not args.no_extras else None
+    sdpa = sdpa_comparator(device) if not args.no_extras else None
+    enc = (encode_measurement(device, with_oracle=(rank == 0 and world == 1 and not args.no_cpu_baseline))
+           if not args.no_extras else None)
     launches = args.steps * T * 2 + 2 * n_enc_steps   # decode + merge kernel per loop step; K and V page encodes
     if rank == 0:
         line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -470,7 +549,7 @@ def run_gpu(args):
                 "scaling": "weak", "vs_baseline": None, "dtype": "u8 codes, f32 accumulate", "data": "synthetic",
                 "config": dict(_config(), parallelism=f"replicas x{world}" if world > 1 else "single GPU"),
                 "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches,
-                "clocks": clocks, "dense_bf16_comparator": dense,
+                "clocks": clocks, "dense_bf16_comparator": dense, "torch_sdpa_bf16": sdpa, "encode": enc,
                 "device_fault_bits": max(status)}
         print(json.dumps(line), flush=True)
     del decode_graphs, encode_graphs
