@@ -324,13 +324,18 @@ LOOPVQ_API size_t loopvq_decode_workspace_bytes(const loopvq_codebook_desc* desc
  *   lse_out                : device [batch][Hq] fp32 natural-log
  *                            log-sum-exp of the scaled scores, or NULL.
  *   workspace              : device, >= loopvq_decode_workspace_bytes, 256-byte
- *                            aligned, ZERO-FILLED before its first use; every
- *                            call leaves it ready for the next one (its split
- *                            counters return to zero) except the status word,
- *                            which only loopvq_clear_device_status resets.
+ *                            aligned, ZERO-FILLED before its first use (it
+ *                            holds the status word and the split partials);
+ *                            only loopvq_clear_device_status resets the
+ *                            status word.
  * Query head hq reads KV head hq / (Hq / H).  A request with ctx_len 0 gets a
  * zero output and lse -inf.  Calls sharing a workspace must be serialised
  * (same stream, or ordered by events).
+ * Each call launches two kernels on `stream`, both as programmatic dependents
+ * of what precedes them: the split kernel (one CTA per split of each request
+ * and query head) and a merge kernel that combines the splits' partials by
+ * log-sum-exp.  The layout's flags, page table, ring window and new-token
+ * inputs are described with loopvq_cache_layout.
  */
 LOOPVQ_API loopvq_status loopvq_decode_attn(const loopvq_codebook_desc* desc, const void* cbK_packed,
                                  const void* cbV_packed, const loopvq_cache_layout* layout,

@@ -139,3 +139,25 @@ def test_dense_rejects_bad_arguments():
               None) == L.LOOPVQ_ERR_INVALID_ARG
     assert dd(1, 16, 16, 128, 100, FAKE, FAKE, 100, FAKE, FAKE, FAKE, 1, 0.1, FAKE, None, FAKE, 64,
               None) == L.LOOPVQ_ERR_WORKSPACE_TOO_SMALL
+
+
+def test_paged_ring_and_new_token_layout_validation():
+    """Paged body, ring window and current-token inputs are validated on the
+    host: an invalid combination gives a zero workspace size."""
+    d = L.make_desc(4, 4, 16, 128, 16)
+    P, R, NT = L.LOOPVQ_LAYOUT_PAGED_BODY, L.LOOPVQ_LAYOUT_RING_WINDOW, L.LOOPVQ_LAYOUT_STATIC_INPUTS
+    paged = dict(flags=P, body_pages=FAKE, body_page_tokens=256, max_body_pages=127, body_off=None)
+    assert L.loopvq_decode_workspace_bytes(d, _layout(**paged)) > 0          # body_off unused when paged
+    assert L.loopvq_decode_workspace_bytes(d, _layout(**dict(paged, max_body_pages=126))) == 0   # too few pages
+    assert L.loopvq_decode_workspace_bytes(d, _layout(**dict(paged, body_page_tokens=48))) == 0  # not a multiple of 32
+    assert L.loopvq_decode_workspace_bytes(d, _layout(**dict(paged, body_page_tokens=36))) == 0
+    assert L.loopvq_decode_workspace_bytes(d, _layout(**dict(paged, body_pages=None))) == 0
+    assert L.loopvq_decode_workspace_bytes(d, _layout(body_off=None)) == 0    # contiguous body needs body_off
+    ring = dict(flags=R | NT, win_head=FAKE, win_ring=264)
+    assert L.loopvq_decode_workspace_bytes(d, _layout(**ring)) > 0
+    assert L.loopvq_decode_workspace_bytes(d, _layout(**dict(ring, win_ring=262))) == 0        # < n_recent + page - 1
+    assert L.loopvq_decode_workspace_bytes(d, _layout(**dict(ring, win_head=None))) == 0
+    assert L.loopvq_decode_workspace_bytes(d, _layout(flags=0x80)) == 0                         # unknown flag
+    assert L.loopvq_decode_workspace_bytes(d, _layout(new_k=FAKE, new_v=FAKE)) > 0
+    assert L.loopvq_decode_workspace_bytes(d, _layout(new_k=FAKE)) == 0                         # K without V
+    assert L.loopvq_decode_workspace_bytes(d, _layout(new_k=FAKE + 2, new_v=FAKE)) == 0         # misaligned
