@@ -50,7 +50,8 @@ WORKLOAD = "ouro1.4b-layer decode attention, batch 1, 16x128, 4 loop steps, Tc=4
 def _config():
     return {"workload": WORKLOAD, "batch": 1, "ctx_len": CTX, "n_heads": H, "head_dim": D, "n_loop": T,
             "tc": TC, "group_elems": G, "bits": 0.5, "n_sink": N_SINK, "n_recent": N_RECENT, "page": PAGE,
-            "step": "4 loop-step decode launches + 8-token page encode (K,V) every 8th step",
+            "step": "4 loop-step decode launches (each stores the new token's bf16 K/V into the window) + "
+                    "8-token page encode (K,V) every 8th step",
             "l2": f"inputs larger than L2: {N_LAYERS} rotating layer caches"}
 
 
@@ -249,11 +250,14 @@ def build_layers(device, n_layers):
     W = G // TC
     J = D // W
     for i in range(n_layers):
-        # the layer's pools and codebooks are not written while its decodes run
-        # (the page encode below writes a separate pool), so the kernel may
-        # start streaming them while the previous launch finishes
+        # the layer's pools, windows and codebooks are not written by other
+        # kernels while its decodes run (the page encode below writes a
+        # separate pool; the new token reaches the window through the
+        # decode's own new_k/new_v write), so a launch may start streaming
+        # them while the previous launch finishes
         c = cache.DecodeCache(n_loop=T, tc=TC, n_heads_kv=H, head_dim=D, group_elems=G, ctx_lens=[CTX],
-                              n_sink=N_SINK, n_recent=N_RECENT, page=PAGE, device=device, static_inputs=True)
+                              n_sink=N_SINK, n_recent=N_RECENT, page=PAGE, device=device, static_inputs=True,
+                              static_windows=True)
         outl = synth.key_outlier_channels(100 + i, H, D)
         c.set_codebooks(synth.uniform_codebook(200 + i, T // TC, H, J, 256, TC, W, outlier_channels=outl),
                         synth.uniform_codebook(300 + i, T // TC, H, J, 256, TC, W))
@@ -262,6 +266,8 @@ def build_layers(device, n_layers):
         c.winK.copy_(synth.device_normal(600 + i, tuple(c.winK.shape), device=device))
         c.winV.copy_(synth.device_normal(700 + i, tuple(c.winV.shape), device=device))
         c.q.copy_(synth.device_normal(800 + i, tuple(c.q.shape), dtype=c.q.dtype, device=device))
+        # the current token's K and V at each loop step, [2][T][batch=1][H][D]
+        c.new_kv = synth.device_normal(850 + i, (2, T, 1, H, D), device=device)
         # the recent page to encode every 8 steps: [T][H][8][D] view of the window pool
         c.page_view = c.winK[:, :, N_SINK:N_SINK + PAGE]
         c.page_view_v = c.winV[:, :, N_SINK:N_SINK + PAGE]
@@ -417,14 +423,14 @@ def run_gpu(args):
     with torch.cuda.stream(stream):
         for c in layers:          # one eager pass (sets attributes, warms caches)
             for t in range(T):
-                c.decode(t, stream=stream)
+                c.decode(t, stream=stream, new_k=c.new_kv[0, t], new_v=c.new_kv[1, t])
             encode_page(c, stream)
     torch.cuda.synchronize()
     for c in layers:
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=stream):
             for t in range(T):
-                c.decode(t, stream=stream)
+                c.decode(t, stream=stream, new_k=c.new_kv[0, t], new_v=c.new_kv[1, t])
         decode_graphs.append(g)
         ge = torch.cuda.CUDAGraph()
         with torch.cuda.graph(ge, stream=stream):
@@ -504,7 +510,8 @@ def run_gpu(args):
         per = []
         for t in range(T):
             lay = L.make_layout(1, N_SINK, N_RECENT, PAGE, c.max_ctx_len, c.ctx_dev, c.body_off_dev, c.win_off_dev,
-                                c.body_pool_tokens, c.win_pool_tokens, L.LOOPVQ_LAYOUT_STATIC_INPUTS,
+                                c.body_pool_tokens, c.win_pool_tokens,
+                                L.LOOPVQ_LAYOUT_STATIC_INPUTS | L.LOOPVQ_LAYOUT_STATIC_WINDOWS,
                                 new_k=k_dev[t], new_v=v_dev[t])
             per.append(L.prepare_decode_attn(c.desc, c.cbK, c.cbV, lay, c.idxK, c.idxV, c.winK, c.winV, q_dev[t], t,
                                              D ** -0.5, out_dev[t], lse_dev[t], c.workspace, stream))

@@ -108,6 +108,10 @@ typedef struct {
 /* The recent tokens live in a ring of win_ring slots per request (see below)
  * instead of right after the sink tokens. */
 #define LOOPVQ_LAYOUT_RING_WINDOW 0x4u
+/* With LOOPVQ_LAYOUT_STATIC_INPUTS: the window pools are not written by the
+ * kernel that precedes the call either (true when the current token arrives
+ * through new_k/new_v), so the window rows are streamed early too. */
+#define LOOPVQ_LAYOUT_STATIC_WINDOWS 0x8u
 
 /*
  * Cache layout of one decode batch.  Request r has ctx_len[r] tokens, the

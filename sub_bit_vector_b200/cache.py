@@ -29,7 +29,7 @@ class DecodeCache:
     def __init__(self, *, n_loop, tc, n_heads_kv, head_dim, group_elems, ctx_lens, n_sink=64, n_recent=256,
                  page=8, n_codes=256, n_heads_q=None, cb_dtype=torch.bfloat16, q_dtype=torch.bfloat16,
                  out_dtype=torch.float32, device="cuda", max_ctx_len=None, pool_slack_tokens=0,
-                 static_inputs=False):
+                 static_inputs=False, static_windows=False):
         self.device = torch.device(device)
         self.T, self.Tc, self.H, self.D, self.G = n_loop, tc, n_heads_kv, head_dim, group_elems
         self.Hq = n_heads_q or n_heads_kv
@@ -72,15 +72,21 @@ class DecodeCache:
         self.body_off_dev = torch.tensor(body_off, dtype=torch.int64, device=dev)
         self.win_off_dev = torch.tensor(win_off, dtype=torch.int64, device=dev)
         # static_inputs: this cache's layout arrays, pools and codebooks are not
-        # written by kernels that may still run when a decode starts
-        self.layout = L.make_layout(self.batch, n_sink, n_recent, page, self.max_ctx_len, self.ctx_dev,
-                                    self.body_off_dev, self.win_off_dev, self.body_pool_tokens,
-                                    self.win_pool_tokens,
-                                    L.LOOPVQ_LAYOUT_STATIC_INPUTS if static_inputs else 0)
+        # written by kernels that may still run when a decode starts;
+        # static_windows: nor its window pools (the current token then comes
+        # through decode(new_k=..., new_v=...))
+        self.flags = ((L.LOOPVQ_LAYOUT_STATIC_INPUTS if static_inputs else 0) |
+                      (L.LOOPVQ_LAYOUT_STATIC_WINDOWS if static_inputs and static_windows else 0))
+        self.layout = self._make_layout(None, None)
         ws = L.loopvq_decode_workspace_bytes(self.desc, self.layout)
         if ws == 0:
             raise ValueError("invalid cache layout")
         self.workspace = torch.zeros(_round_up(ws, 256), dtype=torch.uint8, device=dev)
+
+    def _make_layout(self, new_k, new_v):
+        return L.make_layout(self.batch, self.n_sink, self.n_recent, self.page, self.max_ctx_len, self.ctx_dev,
+                             self.body_off_dev, self.win_off_dev, self.body_pool_tokens, self.win_pool_tokens,
+                             self.flags, new_k=new_k, new_v=new_v)
 
     # ------------------------------------------------------------ inputs
     def set_codebooks(self, cb_k: np.ndarray, cb_v: np.ndarray) -> None:
@@ -120,9 +126,14 @@ class DecodeCache:
         self.q.copy_(torch.from_numpy(np.ascontiguousarray(q, dtype=np.float32)).to(self.device, self.q.dtype))
 
     # ------------------------------------------------------------ compute
-    def decode(self, loop_step: int, softmax_scale: float | None = None, stream=None) -> None:
+    def decode(self, loop_step: int, softmax_scale: float | None = None, stream=None, new_k=None,
+               new_v=None) -> None:
+        """Decode attention at loop_step.  new_k/new_v ([batch][H][D] bf16
+        device tensors) are the current token's K and V at this step: the
+        kernel uses them and stores them in the token's window slot."""
         scale = self.D ** -0.5 if softmax_scale is None else softmax_scale
-        L.loopvq_decode_attn(self.desc, self.cbK, self.cbV, self.layout, self.idxK, self.idxV, self.winK,
+        layout = self.layout if new_k is None else self._make_layout(new_k, new_v)
+        L.loopvq_decode_attn(self.desc, self.cbK, self.cbV, layout, self.idxK, self.idxV, self.winK,
                              self.winV, self.q, loop_step, scale, self.out, self.lse, self.workspace, stream)
 
     def device_status(self):

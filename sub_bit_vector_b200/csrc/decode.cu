@@ -86,6 +86,7 @@ struct DecodeParams {
   int split_len;   // body tokens per split (multiple of 32, <= kSplitCap)
   int max_splits;  // grid.x
   int static_inputs;  // layout arrays, index pools and codebooks are not being written by earlier kernels
+  int static_windows;  // nor the window pools
   // paged body: body token p at pool position body_pages[r][p / bpt] * bpt + p % bpt
   int paged;
   const int32_t* body_pages;
@@ -395,7 +396,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
     const uint8_t* vslice = reinterpret_cast<const uint8_t*>(p.cbV_slice) + (size_t)h * p.C * D * sizeof(CBT);
     const uint32_t vslice_bytes = (uint32_t)(p.C * D * sizeof(CBT));
     if (leader && !is_window && n_tok > 0) prefetch_l2(vslice, vslice_bytes);  // the epilogue's codebook slice
-    if (is_window && p.static_inputs) griddep_wait();  // window rows may come from the previous kernel
+    if (is_window && p.static_inputs && !p.static_windows) griddep_wait();  // rows may come from that kernel
     const int n_slice = (is_window || n_tok == 0) ? 0 : (int)((vslice_bytes + kStageBytes - 1) / kStageBytes);
     const int32_t* pages = p.paged ? p.body_pages + (size_t)r * p.max_body_pages : nullptr;
     const int64_t n_phys = p.paged ? p.body_pool_tokens / p.body_page_tokens : 0;
@@ -811,17 +812,17 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
   // the merge kernel, launched right after as a dependent, combines the splits
 }
 
-// Merge of the splits of every (request, query head): one CTA per unit,
-// launched as a programmatic dependent of the decode kernel (it starts while
-// the decode runs and waits for its completion before reading the
-// partials).  Partials are staged 32 splits at a time, every load of a stage
-// in flight together; the log-sum-exp merge runs online across stages.
-constexpr int kMergeThreads = 256;
+// Merge of the splits of every (request, query head): one CTA of D threads
+// per unit, launched as a programmatic dependent of the decode kernel (it
+// starts while the decode runs and waits for its completion before reading
+// the partials).  Thread d loads column d of up to 32 partial rows at once and
+// lane s of every warp the (m, l) of split s -- one round trip to L2, no
+// shared memory -- and the log-sum-exp weights travel by shuffles; more than
+// 32 splits merge online, 32 at a time.
 constexpr int kMergeChunk = 32;
 
 template <int D>
-__global__ void __launch_bounds__(kMergeThreads) merge_kernel(const DecodeParams p) {
-  __shared__ __align__(16) float sm[kMergeChunk * (D + 4)];
+__global__ void __launch_bounds__(D) merge_kernel(const DecodeParams p) {
   griddep_launch_dependents();
   const int tid = threadIdx.x, lane = tid & 31;
   const int hq = blockIdx.x, r = blockIdx.y;
@@ -833,53 +834,38 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const DecodeParams
   const int n_splits = ctx == 0 ? 0 : (n_win > 0 ? 1 : 0) + (cs.body + p.split_len - 1) / p.split_len;
   griddep_wait();
   const float* part = p.partials + unit * p.max_splits * (size_t)(D + 4);
-  constexpr int kPer = (kMergeChunk * (D + 4) / 4 + kMergeThreads - 1) / kMergeThreads;
-  float M = -INFINITY, Ls = 0.f, o = 0.f;  // running merge; thread d < D holds o[d]
+  float M = -INFINITY, Ls = 0.f, o = 0.f;  // running merge
   for (int c0 = 0; c0 < n_splits; c0 += kMergeChunk) {
     const int nc = min(kMergeChunk, n_splits - c0);
-    const int n4 = nc * (D + 4) / 4;
-    const float4* src = reinterpret_cast<const float4*>(part + (size_t)c0 * (D + 4));
-    float4 v[kPer];
+    const float* rows = part + (size_t)c0 * (D + 4);
+    float ov[kMergeChunk];
 #pragma unroll
-    for (int u = 0; u < kPer; ++u) {
-      const int i = tid + u * kMergeThreads;
-      if (i < n4) v[u] = __ldcg(src + i);
-    }
+    for (int s = 0; s < kMergeChunk; ++s) ov[s] = s < nc ? __ldcg(rows + (size_t)s * (D + 4) + tid) : 0.f;
+    const float ms = lane < nc ? __ldcg(rows + (size_t)lane * (D + 4) + D) : -INFINITY;
+    const float ls = lane < nc ? __ldcg(rows + (size_t)lane * (D + 4) + D + 1) : 0.f;
+    float Mc = ms;
 #pragma unroll
-    for (int u = 0; u < kPer; ++u) {
-      const int i = tid + u * kMergeThreads;
-      if (i < n4) reinterpret_cast<float4*>(sm)[i] = v[u];
-    }
-    __syncthreads();
-    if (tid < D) {
-      const float ms = lane < nc ? sm[lane * (D + 4) + D] : -INFINITY;
-      const float ls = lane < nc ? sm[lane * (D + 4) + D + 1] : 0.f;
-      float Mc = ms;
+    for (int x = 16; x >= 1; x >>= 1) Mc = fmaxf(Mc, __shfl_xor_sync(0xffffffffu, Mc, x));
+    const float Mn = fmaxf(M, Mc);
+    const float e = ms == -INFINITY ? 0.f : exp2f(ms - Mn);
+    float Lc = ls * e;
 #pragma unroll
-      for (int x = 16; x >= 1; x >>= 1) Mc = fmaxf(Mc, __shfl_xor_sync(0xffffffffu, Mc, x));
-      const float Mn = fmaxf(M, Mc);
-      const float e = ms == -INFINITY ? 0.f : exp2f(ms - Mn);
-      float Lc = ls * e;
+    for (int x = 16; x >= 1; x >>= 1) Lc += __shfl_xor_sync(0xffffffffu, Lc, x);
+    const float keep = M == -INFINITY ? 0.f : exp2f(M - Mn);
+    float oc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int x = 16; x >= 1; x >>= 1) Lc += __shfl_xor_sync(0xffffffffu, Lc, x);
-      const float keep = M == -INFINITY ? 0.f : exp2f(M - Mn);
-      float oc[4] = {0.f, 0.f, 0.f, 0.f};
-      for (int s = 0; s < nc; ++s) oc[s & 3] = fmaf(sm[s * (D + 4) + tid], __shfl_sync(0xffffffffu, e, s), oc[s & 3]);
-      o = fmaf(o, keep, (oc[0] + oc[1]) + (oc[2] + oc[3]));
-      Ls = fmaf(Ls, keep, Lc);
-      M = Mn;
-    }
-    __syncthreads();
+    for (int s = 0; s < kMergeChunk; ++s) oc[s & 3] = fmaf(ov[s], __shfl_sync(0xffffffffu, e, s), oc[s & 3]);
+    o = fmaf(o, keep, (oc[0] + oc[1]) + (oc[2] + oc[3]));
+    Ls = fmaf(Ls, keep, Lc);
+    M = Mn;
   }
-  if (tid < D) {
-    const bool ok = M != -INFINITY && Ls > 0.f;
-    const float res = ok ? o * __frcp_rn(Ls) : 0.f;
-    if (p.out_bf16)
-      reinterpret_cast<__nv_bfloat16*>(p.out)[unit * D + tid] = __float2bfloat16_rn(res);
-    else
-      reinterpret_cast<float*>(p.out)[unit * D + tid] = res;
-    if (p.lse && tid == 0) p.lse[unit] = ok ? (M + log2f(Ls)) * 0.6931471805599453f : -INFINITY;
-  }
+  const bool ok = M != -INFINITY && Ls > 0.f;
+  const float res = ok ? o * __frcp_rn(Ls) : 0.f;
+  if (p.out_bf16)
+    reinterpret_cast<__nv_bfloat16*>(p.out)[unit * D + tid] = __float2bfloat16_rn(res);
+  else
+    reinterpret_cast<float*>(p.out)[unit * D + tid] = res;
+  if (p.lse && tid == 0) p.lse[unit] = ok ? (M + log2f(Ls)) * 0.6931471805599453f : -INFINITY;
 }
 
 // Launches the decode kernel as a programmatic dependent of the previous
@@ -938,7 +924,8 @@ static loopvq_status check_layout(const loopvq_cache_layout* L) {
   if (!L || L->batch < 1 || L->n_sink < 0 || L->n_recent < 0 || L->page < 1 || L->max_ctx_len < 0)
     return LOOPVQ_ERR_INVALID_ARG;
   const bool paged = L->flags & LOOPVQ_LAYOUT_PAGED_BODY, ring = L->flags & LOOPVQ_LAYOUT_RING_WINDOW;
-  if (L->flags & ~(LOOPVQ_LAYOUT_STATIC_INPUTS | LOOPVQ_LAYOUT_PAGED_BODY | LOOPVQ_LAYOUT_RING_WINDOW))
+  if (L->flags & ~(LOOPVQ_LAYOUT_STATIC_INPUTS | LOOPVQ_LAYOUT_PAGED_BODY | LOOPVQ_LAYOUT_RING_WINDOW |
+                   LOOPVQ_LAYOUT_STATIC_WINDOWS))
     return LOOPVQ_ERR_INVALID_ARG;
   if (!L->ctx_len || !L->win_off || (!paged && !L->body_off)) return LOOPVQ_ERR_INVALID_ARG;
   if (L->body_pool_tokens < 0 || (L->body_pool_tokens & 31) || L->win_pool_tokens < 0) return LOOPVQ_ERR_INVALID_ARG;
@@ -958,6 +945,7 @@ static loopvq_status check_layout(const loopvq_cache_layout* L) {
 
 // Layout fields of the kernel parameters shared by both entry points.
 static void fill_layout_params(DecodeParams& p, const loopvq_cache_layout* L) {
+  p.static_windows = ((L->flags & LOOPVQ_LAYOUT_STATIC_WINDOWS) && (L->flags & LOOPVQ_LAYOUT_STATIC_INPUTS)) ? 1 : 0;
   p.paged = (L->flags & LOOPVQ_LAYOUT_PAGED_BODY) ? 1 : 0;
   p.body_pages = L->body_pages;
   p.body_page_tokens = p.paged ? L->body_page_tokens : 32;
@@ -1051,7 +1039,7 @@ extern "C" loopvq_status loopvq_decode_attn(const loopvq_codebook_desc* desc, co
     if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, kDynSmem) != cudaSuccess) \
       return LOOPVQ_ERR_CUDA;                                                                        \
     if (launch_pdl((const void*)kfn, grid, s, &p) != cudaSuccess) return LOOPVQ_ERR_CUDA;           \
-    if (launch_pdl((const void*)merge_kernel<DD>, dim3(g.Hq, layout->batch), s, &p, kMergeThreads, 0) != \
+    if (launch_pdl((const void*)merge_kernel<DD>, dim3(g.Hq, layout->batch), s, &p, DD, 0) !=          \
         cudaSuccess)                                                                                 \
       return LOOPVQ_ERR_CUDA;                                                                        \
   } while (0)
@@ -1190,7 +1178,7 @@ extern "C" loopvq_status loopvq_decode_attn_noalloc(const loopvq_codebook_desc* 
     if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, kDynSmem) != cudaSuccess) \
       return LOOPVQ_ERR_CUDA;                                                                        \
     if (launch_pdl((const void*)kfn, grid, s, &p) != cudaSuccess) return LOOPVQ_ERR_CUDA;           \
-    if (launch_pdl((const void*)merge_kernel<DD>, dim3(g.Hq, layout->batch), s, &p, kMergeThreads, 0) != \
+    if (launch_pdl((const void*)merge_kernel<DD>, dim3(g.Hq, layout->batch), s, &p, DD, 0) !=          \
         cudaSuccess)                                                                                 \
       return LOOPVQ_ERR_CUDA;                                                                        \
   } while (0)

@@ -35,6 +35,7 @@ LOOPVQ_FAULT_TIMEOUT = 0x8
 LOOPVQ_LAYOUT_STATIC_INPUTS = 0x1
 LOOPVQ_LAYOUT_PAGED_BODY = 0x2
 LOOPVQ_LAYOUT_RING_WINDOW = 0x4
+LOOPVQ_LAYOUT_STATIC_WINDOWS = 0x8
 
 EXPORTED = [
     "loopvq_version", "loopvq_status_string", "loopvq_validate_desc", "loopvq_ctx_split",
