@@ -64,6 +64,7 @@ __all__ = [
     "kmeans_update",
     "kmeans",
     "distortion",
+    "attention_mse_codebook_grad",
 ]
 
 
@@ -400,3 +401,84 @@ def kmeans(X: np.ndarray, codebook: np.ndarray, tc: int, n_iter: int):
         history.append(distortion(X, idx, cb, tc))
         cb, _ = kmeans_update(X, idx, cb, tc)
     return cb, idx, history
+
+
+# --------------------------------------------------------------------------
+# codebook gradient of the attention-output error (fine-tuning stand-in)
+# --------------------------------------------------------------------------
+# Project page, "Method" -- "Component 2, Loop-aware codebook fine-tuning":
+# the codebooks are tuned so that the quantized model's output matches the
+# full-precision model's while every loop step reads the quantized cache.
+# Without weights or data, the stand-in objective is one attention layer:
+# at loop step t, the squared error between decode attention over the
+# quantized cache and a target output (attention over the full-precision
+# cache), with a weight per step for the steps' unequal sensitivity.  Its
+# gradient with respect to both codebooks follows by the chain rule through
+# softmax attention.
+
+def attention_mse_codebook_grad(q, loop_step, tc, idx_k, idx_v, codebook_k, codebook_v,
+                                win_k, win_v, scale, target, weight=1.0):
+    """Loss and codebook gradients of one request's decode attention at step t.
+
+    L = weight * sum_hq ||o_hq - target_hq||^2 with o from ``decode_attention``
+    (same arguments).  Chain rule, per query head hq reading KV head h over
+    the window and body tokens n with scores s_n = scale q.k_n, softmax
+    weights p_n and o = sum_n p_n v_n:
+
+    * dL/do        g = 2 weight (o - target)
+    * dL/dv_n      p_n g
+    * dL/ds_n      p_n (g.v_n - g.o)   (softmax Jacobian)
+    * dL/dk_n      dL/ds_n * scale * q
+
+    A body token's k_n channels jW+w are codebook entries
+    B^K[b][h][j][idx_k[b][h][n][j]][t - b*Tc][w] (``dequantize``), so each
+    token's dL/dk_n and dL/dv_n slices are added into the entry its code
+    selects; window tokens are stored bf16 and reach no codebook entry.
+
+    target  ``[Hq][D]``; returns ``(loss, grad_k, grad_v, o)`` with the
+    gradients in codebook layout ``[NB][H][J][C][Tc][W]`` (fp64, non-zero
+    only in block b = t // Tc, slice t - b*Tc) and o ``[Hq][D]``.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    target = np.asarray(target, dtype=np.float64)
+    Hq, D = q.shape
+    NB, H, J, C, tc2, w = codebook_k.shape
+    group = Hq // H
+    b, tt = divmod(loop_step, tc)
+    Kb = dequantize(idx_k, codebook_k, loop_step, tc)  # [n_body][H][D]
+    Vb = dequantize(idx_v, codebook_v, loop_step, tc)
+    n_body = Kb.shape[0]
+    grad_k = np.zeros(codebook_k.shape, dtype=np.float64)
+    grad_v = np.zeros(codebook_v.shape, dtype=np.float64)
+    out = np.empty((Hq, D), dtype=np.float64)
+    loss = 0.0
+    for hq in range(Hq):
+        h = hq // group
+        wk = np.asarray(win_k[h], dtype=np.float64)
+        wv = np.asarray(win_v[h], dtype=np.float64)
+        K = np.concatenate([wk, Kb[:, h, :]], axis=0)
+        V = np.concatenate([wv, Vb[:, h, :]], axis=0)
+        if K.shape[0] == 0:
+            out[hq] = 0.0
+            loss += weight * float(np.sum(target[hq] ** 2))
+            continue
+        s = scale * (K @ q[hq])
+        p = np.exp(s - np.max(s))
+        p /= np.sum(p)
+        o = p @ V
+        out[hq] = o
+        diff = o - target[hq]
+        loss += weight * float(diff @ diff)
+        g = 2.0 * weight * diff
+        ds = p * (V @ g - g @ o)
+        nw = wk.shape[0]
+        p_body = p[nw:]
+        ds_body = ds[nw:]
+        for j in range(J):
+            sl = slice(j * w, (j + 1) * w)
+            ck = np.asarray(idx_k[b, h, :n_body, j], dtype=np.int64)
+            cv = np.asarray(idx_v[b, h, :n_body, j], dtype=np.int64)
+            # one row per body token, added into the entry its code selects
+            np.add.at(grad_k[b, h, j, :, tt, :], ck, np.outer(ds_body, scale * q[hq, sl]))
+            np.add.at(grad_v[b, h, j, :, tt, :], cv, np.outer(p_body, g[sl]))
+    return loss, grad_k, grad_v, out

@@ -412,3 +412,90 @@ def test_lloyd_distortion_never_increases():
     _, _, hist = O.kmeans(X, cb, 4, 5)
     assert all(b <= a * (1 + 1e-12) for a, b in zip(hist, hist[1:]))
     assert hist[-1] < hist[0]
+
+
+# ------------------------------------------ codebook gradient (fine-tuning)
+
+def _grad_case(seed, tc, T=4, H=2, Hq=4, D=8, G=4, n_body=7, n_win=3, n_codes=6, C=256):
+    rng = np.random.default_rng(seed)
+    W = G // tc
+    J = D // W
+    NB = T // tc
+    cbk = rng.standard_normal((NB, H, J, C, tc, W))
+    cbv = rng.standard_normal((NB, H, J, C, tc, W))
+    ik = rng.integers(0, n_codes, (NB, H, n_body, J))
+    iv = rng.integers(0, n_codes, (NB, H, n_body, J))
+    wk = rng.standard_normal((H, n_win, D))
+    wv = rng.standard_normal((H, n_win, D))
+    q = rng.standard_normal((Hq, D))
+    target = 0.3 * rng.standard_normal((Hq, D))
+    return cbk, cbv, ik, iv, wk, wv, q, target
+
+
+def _fd_loss(case, tc, t, scale, weight):
+    cbk, cbv, ik, iv, wk, wv, q, target = case
+    o, _ = O.decode_attention(q, t, tc, ik, iv, cbk, cbv, wk, wv, scale)
+    return weight * float(np.sum((o - target) ** 2))
+
+
+@pytest.mark.parametrize("tc,t,n_win", [(2, 3, 3), (4, 2, 3), (1, 1, 0)])
+def test_codebook_grad_matches_central_differences(tc, t, n_win):
+    """Every gradient entry of the codewords in use, in the step's block and
+    slice, equals the central difference of the loss computed through
+    ``decode_attention``; entries of other slices and blocks and of unused
+    codewords move the loss by nothing and are zero."""
+    scale, weight, eps = 0.7, 1.3, 1e-6
+    case = _grad_case(600 + tc, tc, n_win=n_win)
+    cbk, cbv, ik, iv, wk, wv, q, target = case
+    loss, gk, gv, out = O.attention_mse_codebook_grad(q, t, tc, ik, iv, cbk, cbv, wk, wv, scale, target, weight)
+    assert loss == pytest.approx(_fd_loss(case, tc, t, scale, weight), rel=1e-13)
+    np.testing.assert_allclose(out, O.decode_attention(q, t, tc, ik, iv, cbk, cbv, wk, wv, scale)[0], rtol=1e-13)
+    b, tt = divmod(t, tc)
+    NB, H, J, _, _, W = cbk.shape
+    for which, grad in ((0, gk), (1, gv)):
+        cb = case[which]
+        checked = 0
+        for h in range(H):
+            for j in range(J):
+                for c in range(6):
+                    for w in range(W):
+                        e = (b, h, j, c, tt, w)
+                        keep = cb[e]
+                        cb[e] = keep + eps
+                        up = _fd_loss(case, tc, t, scale, weight)
+                        cb[e] = keep - eps
+                        dn = _fd_loss(case, tc, t, scale, weight)
+                        cb[e] = keep
+                        fd = (up - dn) / (2 * eps)
+                        assert grad[e] == pytest.approx(fd, rel=1e-6, abs=1e-8), (which, e)
+                        checked += int(abs(fd) > 1e-6)
+        assert checked > H * J  # the check is not vacuous
+        # other slices / blocks and unused codewords: zero
+        mask = np.zeros(grad.shape, dtype=bool)
+        mask[b, :, :, :6, tt, :] = True
+        assert np.all(grad[~mask] == 0.0)
+        e = (NB - 1 - b, 0, 0, 1, (tt + 1) % tc, 0) if tc > 1 or NB > 1 else (b, 0, 0, 7, tt, 0)
+        keep = cb[e]
+        cb[e] = keep + 1e-3
+        assert _fd_loss(case, tc, t, scale, weight) == _fd_loss(case, tc, t, scale, weight)
+        moved = _fd_loss(case, tc, t, scale, weight)
+        cb[e] = keep
+        assert moved == pytest.approx(loss, rel=1e-14)
+
+
+def test_codebook_grad_zero_at_target_and_empty_body():
+    """Target equal to the output: zero loss and zero gradient.  A context of
+    window tokens only: zero gradient, loss against the window attention."""
+    tc, t, scale = 2, 1, 0.5
+    cbk, cbv, ik, iv, wk, wv, q, _ = _grad_case(610, tc)
+    o, _ = O.decode_attention(q, t, tc, ik, iv, cbk, cbv, wk, wv, scale)
+    loss, gk, gv, _ = O.attention_mse_codebook_grad(q, t, tc, ik, iv, cbk, cbv, wk, wv, scale, o)
+    # (decode_attention divides after the sum: the two outputs differ by rounding)
+    assert loss < 1e-28 and np.max(np.abs(gk)) < 1e-13 and np.max(np.abs(gv)) < 1e-13
+    target = np.ones_like(o)
+    e0k, e0v = ik[:, :, :0], iv[:, :, :0]
+    loss, gk, gv, out = O.attention_mse_codebook_grad(q, t, tc, e0k, e0v, cbk, cbv, wk, wv, scale, target, 2.0)
+    ref = O.dense_decode_attention(q, wk, wv, scale)[0]
+    np.testing.assert_allclose(out, ref, rtol=1e-13)
+    assert loss == pytest.approx(2.0 * float(np.sum((ref - 1.0) ** 2)), rel=1e-13)
+    assert not gk.any() and not gv.any()
