@@ -344,6 +344,60 @@ def sdpa_comparator(device, reps=50):
     return {"us_per_launch": us, "kv_tokens_per_s": CTX / (us * 1e-6), "what": "torch SDPA, bf16 K/V, 1 query"}
 
 
+def all_steps_measurement(layers, device, reps=400):
+    """All T loop steps of a layer in one launch (loopvq_decode_attn_steps):
+    for callers that hold every step's query at once, not loop-sequential
+    decoding.  The steps of one code block share each index row, so a launch
+    moves the codes once and every step's window, query and output."""
+    import torch
+    from sub_bit_vector_b200 import loopvq as L, synth
+    s = torch.cuda.Stream(device)
+    bufs = []
+    for i, c in enumerate(layers):
+        q = synth.device_normal(1700 + i, (T, 1, H, D), device=device)
+        out = torch.zeros((T, 1, H, D), dtype=torch.float32, device=device)
+        lse = torch.zeros((T, 1, H), dtype=torch.float32, device=device)
+        ws = torch.zeros(L.loopvq_decode_steps_workspace_bytes(c.desc, c.layout, T), dtype=torch.uint8,
+                         device=device)
+        bufs.append((c, q, out, lse, ws))
+
+    def launch(b):
+        c, q, out, lse, ws = b
+        L.loopvq_decode_attn_steps(c.desc, c.cbK, c.cbV, c.layout, c.idxK, c.idxV, c.winK, c.winV, q, 0, T,
+                                   D ** -0.5, out, lse, ws, s)
+    with torch.cuda.stream(s):
+        for b in bufs:
+            launch(b)
+    torch.cuda.synchronize()
+    graphs = []
+    for b in bufs:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s):
+            launch(b)
+        graphs.append(g)
+    for i in range(2 * len(graphs)):
+        graphs[i % len(graphs)].replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(s)
+    for i in range(reps):
+        graphs[i % len(graphs)].replay()
+    e1.record(s)
+    torch.cuda.synchronize()
+    us_launch = e0.elapsed_time(e1) * 1e3 / reps
+    faults = max(L.loopvq_read_device_status(b[4])[1] for b in bufs)
+    c = layers[0]
+    per_step = c.algorithmic_bytes()
+    codes = sum(b for (_, b, _) in c.splits) * H * 2 * (D * TC // G)
+    by = codes + T * (per_step - codes)      # codes once, window + q/out per step
+    del graphs
+    return {"us_per_launch": us_launch, "us_per_loop_step": us_launch / T,
+            "kv_tokens_per_s_per_step": CTX * T / (us_launch * 1e-6), "algorithmic_bytes_per_launch": by,
+            "GB_per_s": by / us_launch / 1e3, "launches_timed": reps, "device_fault_bits": faults,
+            "what": f"{T} loop steps per launch (every step's query given at once), graph of 1 launch per layer, "
+                    f"{len(layers)} rotating layer caches"}
+
+
 def encode_measurement(device, with_oracle, reps=5):
     """Loop-axis encode of a 32768-token prefill's keys [4][32768][16][128]
     bf16 at 0.5 bit (tensor-core kernel); with_oracle adds the oracle's rate
@@ -545,6 +599,7 @@ def run_gpu(args):
                    "also write the new token into the window (+ page encode every 8th step), fp32 outputs -> "
                    "pinned host, stream sync per step"}
 
+    steps_fused = all_steps_measurement(layers, device) if not args.no_extras else None
     dense = dense_comparator(device) if not args.no_extras else None
     sdpa = sdpa_comparator(device) if not args.no_extras else None
     enc = (encode_measurement(device, with_oracle=(rank == 0 and world == 1 and not args.no_cpu_baseline))
@@ -556,7 +611,7 @@ def run_gpu(args):
                 "scaling": "weak", "vs_baseline": None, "dtype": "u8 codes, f32 accumulate", "data": "synthetic",
                 "config": dict(_config(), parallelism=f"replicas x{world}" if world > 1 else "single GPU"),
                 "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches,
-                "clocks": clocks, "dense_bf16_comparator": dense, "torch_sdpa_bf16": sdpa, "encode": enc,
+                "clocks": clocks, "all_steps_one_launch": steps_fused, "dense_bf16_comparator": dense, "torch_sdpa_bf16": sdpa, "encode": enc,
                 "device_fault_bits": max(status)}
         print(json.dumps(line), flush=True)
     del decode_graphs, encode_graphs

@@ -351,6 +351,37 @@ LOOPVQ_API loopvq_status loopvq_decode_attn(const loopvq_codebook_desc* desc, co
                                  loopvq_stream_t stream);
 
 /*
+ * Several loop steps of one decode in a single launch: steps first_step ..
+ * first_step + n_steps - 1, for a caller that has every step's query at once
+ * (a fused all-steps decode).  This is not loop-sequential decoding, where
+ * step t+1's query is computed from step t's output and each step is its own
+ * loopvq_decode_attn call.  Step t of the launch computes exactly what
+ * loopvq_decode_attn(loop_step = t) computes; the split kernel places the
+ * CTAs of the n_steps steps that share a (query head, split) next to each
+ * other, so the steps of one code block read each index row from HBM once
+ * and from L2 after that.
+ *   q            : device [n_steps][batch][Hq][D] in q_dtype.
+ *   out, lse_out : device [n_steps][batch][Hq][D] and [n_steps][batch][Hq]
+ *                  (lse_out may be NULL).
+ *   workspace    : >= loopvq_decode_steps_workspace_bytes(desc, layout,
+ *                  n_steps) bytes, as for loopvq_decode_attn.
+ *   layout->new_k, new_v : if given, device bf16 [n_steps][batch][H][D], the
+ *                  current token's K and V at each of the steps.
+ * Everything else is as for loopvq_decode_attn; 1 <= n_steps and
+ * first_step + n_steps <= n_loop.
+ */
+LOOPVQ_API size_t loopvq_decode_steps_workspace_bytes(const loopvq_codebook_desc* desc,
+                                                      const loopvq_cache_layout* layout, int32_t n_steps);
+LOOPVQ_API loopvq_status loopvq_decode_attn_steps(const loopvq_codebook_desc* desc, const void* cbK_packed,
+                                                  const void* cbV_packed, const loopvq_cache_layout* layout,
+                                                  const uint8_t* idxK_pool, const uint8_t* idxV_pool,
+                                                  const void* winK, const void* winV, const void* q,
+                                                  loopvq_dtype q_dtype, int32_t first_step, int32_t n_steps,
+                                                  float softmax_scale, void* out, loopvq_dtype out_dtype,
+                                                  float* lse_out, void* workspace, size_t workspace_bytes,
+                                                  loopvq_stream_t stream);
+
+/*
  * Allocation-free variant of loopvq_decode_attn (the LoopVQ pages have no
  * counterpart; this is a packaging choice of the library).
  *
@@ -389,6 +420,53 @@ LOOPVQ_API loopvq_status loopvq_read_device_status(const void* workspace, uint32
 
 /* Zeroes the status word (asynchronously on stream). */
 LOOPVQ_API loopvq_status loopvq_clear_device_status(void* workspace, loopvq_stream_t stream);
+
+/* ------------------------------------- codebook gradient (fine-tuning) */
+
+/*
+ * Gradients of the decode-attention output error with respect to both
+ * codebooks: the stand-in objective for loop-aware codebook fine-tuning
+ * (project page, "Method" -- "Component 2, Loop-aware codebook fine-tuning":
+ * codebooks tuned so that the quantized model's output matches the
+ * full-precision one while every loop step reads the quantized cache).  At
+ * loop step t,
+ *   L = weight * sum_{request r, query head hq} || out[r][hq] - target[r][hq] ||^2
+ * where out is loopvq_decode_attn's fp32 output of the same step, layout,
+ * codes and queries, and target is, e.g., attention over the full-precision
+ * cache (a per-step weight models the steps' unequal sensitivity).  With
+ * g = 2 weight (o - target) and p_n = exp(s_n - lse) the softmax weight of
+ * body token n, the call ADDS
+ *   gradV[b][h][j][c][t-b*Tc][w] += sum_{n: idxV[n][j]=c} p_n g[j*W+w]
+ *   gradK[b][h][j][c][t-b*Tc][w] += sum_{n: idxK[n][j]=c} p_n (g.v_n - g.o) scale q[j*W+w]
+ * (b = t / Tc; other blocks and slices are untouched) and, if loss_out is
+ * non-NULL, adds L to *loss_out.  Window tokens are bf16 and reach no
+ * codebook entry (they act only through out and lse), so winK/winV are not
+ * read.  Several requests of the layout may share one cache (equal body_off
+ * or page tables): the gradient is then summed over their queries.
+ *   cbK, cbV       : device, CANONICAL layout [NB][H][J][C][Tc][W] in
+ *                    desc->cb_dtype (the values the forward's packed
+ *                    codebooks were made from).
+ *   layout, idxK_pool, idxV_pool, q, q_dtype, loop_step, softmax_scale : as
+ *                    given to loopvq_decode_attn.
+ *   out            : device fp32 [batch][Hq][D], the forward's output.
+ *   lse            : device fp32 [batch][Hq], the forward's lse_out.
+ *   target         : device fp32 [batch][Hq][D].
+ *   gradK, gradV   : device fp32, canonical layout, accumulated into (the
+ *                    caller zeroes them).
+ *   loss_out       : device fp32 scalar, accumulated into, or NULL.
+ *   fault_bits     : device uint32 receiving LOOPVQ_FAULT_* bits (a code
+ *                    >= n_codes: that token is skipped; a context or pool
+ *                    out of range: that request is skipped), or NULL.
+ * J must be 8, 16 or 32 and D 64 or 128.  One kernel on `stream`; sums use
+ * fp32 atomics, so results are reproducible only up to rounding order.
+ */
+LOOPVQ_API loopvq_status loopvq_codebook_grad(const loopvq_codebook_desc* desc, const void* cbK, const void* cbV,
+                                              const loopvq_cache_layout* layout, const uint8_t* idxK_pool,
+                                              const uint8_t* idxV_pool, const void* q, loopvq_dtype q_dtype,
+                                              int32_t loop_step, float softmax_scale, const float* out,
+                                              const float* lse, const float* target, float weight,
+                                              float* gradK, float* gradV, float* loss_out,
+                                              uint32_t* fault_bits, loopvq_stream_t stream);
 
 /* -------------------------------------------------- dense bf16 comparator */
 

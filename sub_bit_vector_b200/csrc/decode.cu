@@ -83,6 +83,12 @@ struct DecodeParams {
   uint32_t* status;
   uint32_t* tickets;
   float* partials;
+  // Several loop steps in one launch: step loop_step + i for i < n_steps;
+  // queries, outputs, lse and partials are [n_steps][batch][Hq]..., the
+  // codebook slices and window pools advance by a step's size, the index
+  // pools by a code block's.
+  int n_steps;
+  int64_t slice_step_elems, win_step_elems, idx_blk_bytes;
   int split_len;   // body tokens per split (multiple of 32, <= kSplitCap)
   int max_splits;  // grid.x
   int static_inputs;  // layout arrays, index pools and codebooks are not being written by earlier kernels
@@ -273,14 +279,20 @@ __device__ __forceinline__ float load_q(const void* q, int q_bf16, size_t i) {
                 : reinterpret_cast<const float*>(q)[i];
 }
 
-template <int J, int D, typename CBT>
+// kSteps: a launch of several loop steps (the single-step instance keeps the
+// step index a compile-time zero and its registers to itself).
+template <int J, int D, typename CBT, bool kSteps>
 __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams p) {
   extern __shared__ __align__(1024) uint8_t dyn[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   // Query head fastest, the window split last: CTAs are dispatched in this
   // order, so the light window splits take the SMs that the previous launch
   // frees last and every body split starts (and prefetches) as early as it can.
-  const int hq = blockIdx.x, split = blockIdx.y, r = blockIdx.z;
+  // The steps of one (query head, split) are adjacent in x, so they run side
+  // by side and share each index row through L2.
+  const int hq = kSteps ? (int)(blockIdx.x / p.n_steps) : (int)blockIdx.x;
+  const int split = blockIdx.y, r = blockIdx.z;
+  auto step_index = [&]() -> int { return kSteps ? (int)(blockIdx.x - (blockIdx.x / p.n_steps) * p.n_steps) : 0; };
   const int group = p.Hq / p.H;
   const int h = hq / group;
   constexpr int W = D / J;
@@ -293,7 +305,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
   int ctx = __ldg(p.ctx_len + r);
   const int64_t body_off = __ldg(p.body_off + r);
   const int64_t win_off = __ldg(p.win_off + r);
-  const size_t unit = (size_t)r * p.Hq + hq;
+  const size_t unit = ((size_t)step_index() * p.batch + r) * p.Hq + hq;
   // The query row is read right after the dependency resolves; pulling its
   // lines into L2 now (a hint: L2 stays coherent with the previous kernel's
   // writes) takes the DRAM latency off that critical step.
@@ -302,7 +314,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
     asm volatile("prefetch.global.L2 [%0];" ::"l"(qrow + tid * 128));
   }
   float wk[kPer][W];               // B^K_t entries (c, j) = tid + 512k, code-major slice
-  const CBT* bk = reinterpret_cast<const CBT*>(p.cbK_slice) + (size_t)h * p.C * J * W;
+  const CBT* bk = reinterpret_cast<const CBT*>(p.cbK_slice) + step_index() * p.slice_step_elems + (size_t)h * p.C * J * W;
   if (tid < kNW * 32) {
 #pragma unroll
     for (int k = 0; k < kPer; ++k) {
@@ -393,7 +405,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
   // the paged body); lane 0 issues the barrier operations and the copies.
   if (warp == kNW) {
     const bool leader = lane == 0;
-    const uint8_t* vslice = reinterpret_cast<const uint8_t*>(p.cbV_slice) + (size_t)h * p.C * D * sizeof(CBT);
+    const int sidx = step_index();
+    const uint8_t* vslice = reinterpret_cast<const uint8_t*>(p.cbV_slice) +
+                            (sidx * p.slice_step_elems + (size_t)h * p.C * D) * sizeof(CBT);
+    const int64_t idx_blk = (int64_t)((p.loop_step + sidx) / p.Tc - p.loop_step / p.Tc) * p.idx_blk_bytes;
     const uint32_t vslice_bytes = (uint32_t)(p.C * D * sizeof(CBT));
     if (leader && !is_window && n_tok > 0) prefetch_l2(vslice, vslice_bytes);  // the epilogue's codebook slice
     if (is_window && p.static_inputs && !p.static_windows) griddep_wait();  // rows may come from that kernel
@@ -425,7 +440,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
         const bool vpass = k >= n_chunks_half;
         const int t0 = (vpass ? k - n_chunks_half : k) * kRowsPerChunk;
         const int t1 = min(n_tok, t0 + kRowsPerChunk);
-        const __nv_bfloat16* base = (vpass ? p.winV : p.winK) + (size_t)h * p.win_pool_tokens * D;
+        const __nv_bfloat16* base = (vpass ? p.winV : p.winK) + sidx * p.win_step_elems + (size_t)h * p.win_pool_tokens * D;
         if (leader) {
           mbar_arrive_expect_tx(fb, (uint32_t)(t1 - t0) * D * 2);
           for (int i = t0; i < t1;) {  // contiguous runs of rows (a ring wraps once at most)
@@ -440,7 +455,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
         const int c = vpass ? k - n_chunks_half : k;
         const int tl0 = c * kTilesPerChunk;
         const int nt = min(kTilesPerChunk, n_tiles - tl0);
-        const uint8_t* stream = (vpass ? p.idxV : p.idxK) + (int64_t)h * (p.body_pool_tokens >> 5) * (32 * J);
+        const uint8_t* stream = (vpass ? p.idxV : p.idxK) + idx_blk + (int64_t)h * (p.body_pool_tokens >> 5) * (32 * J);
         if (!p.paged) {
           if (leader) {
             const int64_t tile = ((body_off + tok0) >> 5) + tl0;
@@ -503,10 +518,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
     const bool has_new = p.new_k != nullptr && n_tok > 0;
     if (has_new && hq % group == 0 && warp == 0) {
       const int64_t row = win_row(p, win_off, cs.sink, whead, i_cur);
-      const size_t src = ((size_t)r * p.H + h) * D + lane * CPL;
+      const int sidx = step_index();
+      const size_t src = (((size_t)sidx * p.batch + r) * p.H + h) * D + lane * CPL;
       const size_t dstp = ((size_t)h * p.win_pool_tokens + row) * D + lane * CPL;
-      __nv_bfloat16* wk = const_cast<__nv_bfloat16*>(p.winK);
-      __nv_bfloat16* wv = const_cast<__nv_bfloat16*>(p.winV);
+      __nv_bfloat16* wk = const_cast<__nv_bfloat16*>(p.winK) + sidx * p.win_step_elems;
+      __nv_bfloat16* wv = const_cast<__nv_bfloat16*>(p.winV) + sidx * p.win_step_elems;
 #pragma unroll
       for (int i = 0; i < CPL; ++i) {
         wk[dstp + i] = p.new_k[src + i];
@@ -516,7 +532,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
     // overwrite row i_cur - t0 of a stage that holds window tokens from t0
     auto patch_row = [&](uint8_t* st, int t0, const __nv_bfloat16* nv) {
       if (warp == 0) {
-        const __nv_bfloat16* src = nv + ((size_t)r * p.H + h) * D + lane * CPL;
+        const __nv_bfloat16* src = nv + (((size_t)step_index() * p.batch + r) * p.H + h) * D + lane * CPL;
         __nv_bfloat16* d = reinterpret_cast<__nv_bfloat16*>(st + (size_t)(i_cur - t0) * D * 2) + lane * CPL;
 #pragma unroll
         for (int i = 0; i < CPL; ++i) d[i] = src[i];
@@ -826,7 +842,7 @@ __global__ void __launch_bounds__(D) merge_kernel(const DecodeParams p) {
   griddep_launch_dependents();
   const int tid = threadIdx.x, lane = tid & 31;
   const int hq = blockIdx.x, r = blockIdx.y;
-  const size_t unit = (size_t)r * p.Hq + hq;
+  const size_t unit = ((size_t)blockIdx.z * p.batch + r) * p.Hq + hq;  // z: step of a multi-step launch
   int ctx = __ldg(p.ctx_len + r);
   if (ctx < 0 || ctx > p.max_ctx) ctx = 0;  // reported by the decode kernel
   const CtxSplit cs = ctx_split(ctx, p.n_sink, p.n_recent, p.page);
@@ -914,8 +930,8 @@ static int max_body_tokens(const loopvq_cache_layout* L) {
 }
 
 // workspace bound independent of the device: plan with a generous SM count
-static WsLayout decode_ws(const Geo& g, const loopvq_cache_layout* L) {
-  const int64_t units = (int64_t)L->batch * g.Hq;
+static WsLayout decode_ws(const Geo& g, const loopvq_cache_layout* L, int n_steps = 1) {
+  const int64_t units = (int64_t)L->batch * g.Hq * n_steps;
   DecodePlan pl = decode_plan(units, max_body_tokens(L), 1024);
   return ws_layout(units, pl.max_splits, g.D);
 }
@@ -961,86 +977,81 @@ static void fill_layout_params(DecodeParams& p, const loopvq_cache_layout* L) {
 
 using namespace loopvq;
 
-extern "C" size_t loopvq_decode_workspace_bytes(const loopvq_codebook_desc* desc,
-                                                const loopvq_cache_layout* layout) {
-  Geo g;
-  if (make_geo(desc, &g) != LOOPVQ_OK || check_layout(layout) != LOOPVQ_OK) return 0;
-  return decode_ws(g, layout).total;
-}
+namespace loopvq {
 
-extern "C" loopvq_status loopvq_decode_attn(const loopvq_codebook_desc* desc, const void* cbK_packed,
-                                            const void* cbV_packed, const loopvq_cache_layout* layout,
-                                            const uint8_t* idxK_pool, const uint8_t* idxV_pool,
-                                            const void* winK, const void* winV, const void* q,
-                                            loopvq_dtype q_dtype, int32_t loop_step, float softmax_scale,
-                                            void* out, loopvq_dtype out_dtype, float* lse_out,
-                                            void* workspace, size_t workspace_bytes,
-                                            loopvq_stream_t stream) {
+// Checks the arguments shared by the decode entry points and fills the kernel
+// parameters for steps first_step .. first_step + n_steps - 1 (all but the
+// workspace pointers).
+static loopvq_status decode_setup(const loopvq_codebook_desc* desc, const void* cbK_packed, const void* cbV_packed,
+                                  const loopvq_cache_layout* layout, const uint8_t* idxK_pool,
+                                  const uint8_t* idxV_pool, const void* winK, const void* winV, const void* q,
+                                  loopvq_dtype q_dtype, int32_t first_step, int32_t n_steps, float softmax_scale,
+                                  void* out, loopvq_dtype out_dtype, float* lse_out, Geo* g_out,
+                                  DecodeParams* p_out) {
   Geo g;
   loopvq_status st = make_geo(desc, &g);
   if (st != LOOPVQ_OK) return st;
   if ((st = check_layout(layout)) != LOOPVQ_OK) return st;
   if (g.J != 8 && g.J != 16 && g.J != 32) return LOOPVQ_ERR_UNSUPPORTED;
   if (g.D != 64 && g.D != 128) return LOOPVQ_ERR_UNSUPPORTED;
-  if (loop_step < 0 || loop_step >= g.T) return LOOPVQ_ERR_INVALID_ARG;
+  if (n_steps < 1 || first_step < 0 || first_step > g.T - n_steps) return LOOPVQ_ERR_INVALID_ARG;
   if (q_dtype != LOOPVQ_F32 && q_dtype != LOOPVQ_BF16) return LOOPVQ_ERR_INVALID_ARG;
   if (out_dtype != LOOPVQ_F32 && out_dtype != LOOPVQ_BF16) return LOOPVQ_ERR_INVALID_ARG;
   if (!(softmax_scale == softmax_scale)) return LOOPVQ_ERR_INVALID_ARG;
-  if (!cbK_packed || !cbV_packed || !idxK_pool || !idxV_pool || !winK || !winV || !q || !out || !workspace)
+  if (!cbK_packed || !cbV_packed || !idxK_pool || !idxV_pool || !winK || !winV || !q || !out)
     return LOOPVQ_ERR_INVALID_ARG;
   if (((uintptr_t)idxK_pool & 15) || ((uintptr_t)idxV_pool & 15) || ((uintptr_t)winK & 15) ||
-      ((uintptr_t)winV & 15) || ((uintptr_t)workspace & 255) || ((uintptr_t)cbK_packed & 15) ||
-      ((uintptr_t)cbV_packed & 15))
+      ((uintptr_t)winV & 15) || ((uintptr_t)cbK_packed & 15) || ((uintptr_t)cbV_packed & 15))
     return LOOPVQ_ERR_INVALID_ARG;
-  const WsLayout ws = decode_ws(g, layout);
-  if (workspace_bytes < ws.total) return LOOPVQ_ERR_WORKSPACE_TOO_SMALL;
-
-  const int64_t units = (int64_t)layout->batch * g.Hq;
+  const int64_t units = (int64_t)layout->batch * g.Hq * n_steps;
   const DecodePlan pl = decode_plan(units, max_body_tokens(layout), device_sm_count());
-  if (units > 65535LL * 65535LL || pl.max_splits > kMaxCombineSplits || layout->batch > 65535 || g.Hq > 65535)
+  if (units > 65535LL * 65535LL || pl.max_splits > kMaxCombineSplits || layout->batch > 65535 ||
+      (int64_t)g.Hq * n_steps > 65535)
     return LOOPVQ_ERR_UNSUPPORTED;
 
-  DecodeParams p;
+  DecodeParams& p = *p_out;
   p.T = g.T; p.Tc = g.Tc; p.H = g.H; p.Hq = g.Hq; p.D = g.D; p.J = g.J; p.W = g.W; p.C = g.C;
-  p.loop_step = loop_step;
+  p.loop_step = first_step;
   p.scale_log2 = softmax_scale * 1.4426950408889634f;
   p.batch = layout->batch; p.n_sink = layout->n_sink; p.n_recent = layout->n_recent;
   p.page = layout->page; p.max_ctx = layout->max_ctx_len;
   p.ctx_len = layout->ctx_len; p.body_off = layout->body_off; p.win_off = layout->win_off;
   p.body_pool_tokens = layout->body_pool_tokens; p.win_pool_tokens = layout->win_pool_tokens;
   const size_t eb = cb_elem_bytes(g);
-  const size_t slices = packed_slices_offset_bytes(g);
-  const size_t step_off = slices + (size_t)loop_step * slice_elems_per_step(g) * eb;
+  const size_t step_off = packed_slices_offset_bytes(g) + (size_t)first_step * slice_elems_per_step(g) * eb;
   p.cbK_slice = (const uint8_t*)cbK_packed + step_off;
   p.cbV_slice = (const uint8_t*)cbV_packed + step_off;
-  const int b_blk = loop_step / g.Tc;
   const size_t blk_bytes = (size_t)g.H * layout->body_pool_tokens * g.J;
-  p.idxK = idxK_pool + b_blk * blk_bytes;
-  p.idxV = idxV_pool + b_blk * blk_bytes;
+  p.idxK = idxK_pool + (first_step / g.Tc) * blk_bytes;
+  p.idxV = idxV_pool + (first_step / g.Tc) * blk_bytes;
   const size_t win_step = (size_t)g.H * layout->win_pool_tokens * g.D;
-  p.winK = (const __nv_bfloat16*)winK + loop_step * win_step;
-  p.winV = (const __nv_bfloat16*)winV + loop_step * win_step;
+  p.winK = (const __nv_bfloat16*)winK + first_step * win_step;
+  p.winV = (const __nv_bfloat16*)winV + first_step * win_step;
   p.q = q; p.q_bf16 = q_dtype == LOOPVQ_BF16;
   p.out = out; p.out_bf16 = out_dtype == LOOPVQ_BF16; p.lse = lse_out;
-  p.status = (uint32_t*)workspace;
-  p.tickets = (uint32_t*)((uint8_t*)workspace + ws.tickets_off);
-  p.partials = (float*)((uint8_t*)workspace + ws.partials_off);
+  p.n_steps = n_steps;
+  p.slice_step_elems = (int64_t)slice_elems_per_step(g);
+  p.win_step_elems = (int64_t)win_step;
+  p.idx_blk_bytes = (int64_t)blk_bytes;
   p.split_len = pl.split_len;
   p.max_splits = pl.max_splits;
-
   p.static_inputs = (layout->flags & LOOPVQ_LAYOUT_STATIC_INPUTS) ? 1 : 0;
   fill_layout_params(p, layout);
+  *g_out = g;
+  return LOOPVQ_OK;
+}
 
-  dim3 grid(g.Hq, pl.max_splits, layout->batch);
-  cudaStream_t s = (cudaStream_t)stream;
+// The split kernel and its dependent merge kernel on `s`.
+static loopvq_status decode_launch(const Geo& g, DecodeParams& p, cudaStream_t s) {
+  const dim3 grid(g.Hq * p.n_steps, p.max_splits, p.batch);
+  const dim3 mgrid(g.Hq, p.batch, p.n_steps);
 #define LOOPVQ_LAUNCH(JJ, DD, CBT)                                                                    \
   do {                                                                                               \
-    auto kfn = decode_kernel<JJ, DD, CBT>;                                                           \
+    auto kfn = p.n_steps > 1 ? decode_kernel<JJ, DD, CBT, true> : decode_kernel<JJ, DD, CBT, false>; \
     if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, kDynSmem) != cudaSuccess) \
       return LOOPVQ_ERR_CUDA;                                                                        \
     if (launch_pdl((const void*)kfn, grid, s, &p) != cudaSuccess) return LOOPVQ_ERR_CUDA;           \
-    if (launch_pdl((const void*)merge_kernel<DD>, dim3(g.Hq, layout->batch), s, &p, DD, 0) !=          \
-        cudaSuccess)                                                                                 \
+    if (launch_pdl((const void*)merge_kernel<DD>, mgrid, s, &p, DD, 0) != cudaSuccess)               \
       return LOOPVQ_ERR_CUDA;                                                                        \
   } while (0)
 #define LOOPVQ_LAUNCH_J(DD, CBT)                      \
@@ -1059,6 +1070,67 @@ extern "C" loopvq_status loopvq_decode_attn(const loopvq_codebook_desc* desc, co
 #undef LOOPVQ_LAUNCH_J
 #undef LOOPVQ_LAUNCH
   return cudaGetLastError() == cudaSuccess ? LOOPVQ_OK : LOOPVQ_ERR_CUDA;
+}
+
+static loopvq_status decode_with_workspace(const loopvq_codebook_desc* desc, const void* cbK_packed,
+                                           const void* cbV_packed, const loopvq_cache_layout* layout,
+                                           const uint8_t* idxK_pool, const uint8_t* idxV_pool, const void* winK,
+                                           const void* winV, const void* q, loopvq_dtype q_dtype,
+                                           int32_t first_step, int32_t n_steps, float softmax_scale, void* out,
+                                           loopvq_dtype out_dtype, float* lse_out, void* workspace,
+                                           size_t workspace_bytes, loopvq_stream_t stream) {
+  Geo g;
+  DecodeParams p;
+  loopvq_status st = decode_setup(desc, cbK_packed, cbV_packed, layout, idxK_pool, idxV_pool, winK, winV, q,
+                                  q_dtype, first_step, n_steps, softmax_scale, out, out_dtype, lse_out, &g, &p);
+  if (st != LOOPVQ_OK) return st;
+  if (!workspace || ((uintptr_t)workspace & 255)) return LOOPVQ_ERR_INVALID_ARG;
+  const WsLayout ws = decode_ws(g, layout, n_steps);
+  if (workspace_bytes < ws.total) return LOOPVQ_ERR_WORKSPACE_TOO_SMALL;
+  p.status = (uint32_t*)workspace;
+  p.tickets = (uint32_t*)((uint8_t*)workspace + ws.tickets_off);
+  p.partials = (float*)((uint8_t*)workspace + ws.partials_off);
+  return decode_launch(g, p, (cudaStream_t)stream);
+}
+
+}  // namespace loopvq
+
+extern "C" size_t loopvq_decode_workspace_bytes(const loopvq_codebook_desc* desc,
+                                                const loopvq_cache_layout* layout) {
+  return loopvq_decode_steps_workspace_bytes(desc, layout, 1);
+}
+
+extern "C" size_t loopvq_decode_steps_workspace_bytes(const loopvq_codebook_desc* desc,
+                                                      const loopvq_cache_layout* layout, int32_t n_steps) {
+  Geo g;
+  if (make_geo(desc, &g) != LOOPVQ_OK || check_layout(layout) != LOOPVQ_OK || n_steps < 1 || n_steps > g.T) return 0;
+  return decode_ws(g, layout, n_steps).total;
+}
+
+extern "C" loopvq_status loopvq_decode_attn(const loopvq_codebook_desc* desc, const void* cbK_packed,
+                                            const void* cbV_packed, const loopvq_cache_layout* layout,
+                                            const uint8_t* idxK_pool, const uint8_t* idxV_pool,
+                                            const void* winK, const void* winV, const void* q,
+                                            loopvq_dtype q_dtype, int32_t loop_step, float softmax_scale,
+                                            void* out, loopvq_dtype out_dtype, float* lse_out,
+                                            void* workspace, size_t workspace_bytes,
+                                            loopvq_stream_t stream) {
+  return decode_with_workspace(desc, cbK_packed, cbV_packed, layout, idxK_pool, idxV_pool, winK, winV, q, q_dtype,
+                               loop_step, 1, softmax_scale, out, out_dtype, lse_out, workspace, workspace_bytes,
+                               stream);
+}
+
+extern "C" loopvq_status loopvq_decode_attn_steps(const loopvq_codebook_desc* desc, const void* cbK_packed,
+                                                  const void* cbV_packed, const loopvq_cache_layout* layout,
+                                                  const uint8_t* idxK_pool, const uint8_t* idxV_pool,
+                                                  const void* winK, const void* winV, const void* q,
+                                                  loopvq_dtype q_dtype, int32_t first_step, int32_t n_steps,
+                                                  float softmax_scale, void* out, loopvq_dtype out_dtype,
+                                                  float* lse_out, void* workspace, size_t workspace_bytes,
+                                                  loopvq_stream_t stream) {
+  return decode_with_workspace(desc, cbK_packed, cbV_packed, layout, idxK_pool, idxV_pool, winK, winV, q, q_dtype,
+                               first_step, n_steps, softmax_scale, out, out_dtype, lse_out, workspace,
+                               workspace_bytes, stream);
 }
 
 // ---------------------------------------------------------------------------
@@ -1114,88 +1186,21 @@ extern "C" loopvq_status loopvq_decode_attn_noalloc(const loopvq_codebook_desc* 
                                                     void* out, loopvq_dtype out_dtype, float* lse_out,
                                                     uint32_t* fault_bits, loopvq_stream_t stream) {
   Geo g;
-  loopvq_status st = make_geo(desc, &g);
+  DecodeParams p;
+  loopvq_status st = decode_setup(desc, cbK_packed, cbV_packed, layout, idxK_pool, idxV_pool, winK, winV, q,
+                                  q_dtype, loop_step, 1, softmax_scale, out, out_dtype, lse_out, &g, &p);
   if (st != LOOPVQ_OK) return st;
-  if ((st = check_layout(layout)) != LOOPVQ_OK) return st;
-  if (g.J != 8 && g.J != 16 && g.J != 32) return LOOPVQ_ERR_UNSUPPORTED;
-  if (g.D != 64 && g.D != 128) return LOOPVQ_ERR_UNSUPPORTED;
-  if (loop_step < 0 || loop_step >= g.T) return LOOPVQ_ERR_INVALID_ARG;
-  if (q_dtype != LOOPVQ_F32 && q_dtype != LOOPVQ_BF16) return LOOPVQ_ERR_INVALID_ARG;
-  if (out_dtype != LOOPVQ_F32 && out_dtype != LOOPVQ_BF16) return LOOPVQ_ERR_INVALID_ARG;
-  if (!(softmax_scale == softmax_scale)) return LOOPVQ_ERR_INVALID_ARG;
-  if (!cbK_packed || !cbV_packed || !idxK_pool || !idxV_pool || !winK || !winV || !q || !out)
-    return LOOPVQ_ERR_INVALID_ARG;
-  if (((uintptr_t)idxK_pool & 15) || ((uintptr_t)idxV_pool & 15) || ((uintptr_t)winK & 15) ||
-      ((uintptr_t)winV & 15) || ((uintptr_t)cbK_packed & 15) || ((uintptr_t)cbV_packed & 15) ||
-      ((uintptr_t)fault_bits & 3))
-    return LOOPVQ_ERR_INVALID_ARG;
+  if ((uintptr_t)fault_bits & 3) return LOOPVQ_ERR_INVALID_ARG;
   const WsLayout ws = decode_ws(g, layout);
   if (ws.total > kLoopvqStaticScratchBytes) return LOOPVQ_ERR_WORKSPACE_TOO_SMALL;
-  const int64_t units = (int64_t)layout->batch * g.Hq;
-  const DecodePlan pl = decode_plan(units, max_body_tokens(layout), device_sm_count());
-  if (units > 65535LL * 65535LL || pl.max_splits > kMaxCombineSplits || layout->batch > 65535 || g.Hq > 65535)
-    return LOOPVQ_ERR_UNSUPPORTED;
 
   void* scratch = nullptr;
   if ((st = static_scratch(&scratch)) != LOOPVQ_OK) return st;
   cudaStream_t s = (cudaStream_t)stream;
   // the status word and the split counters must start at zero
   if (cudaMemsetAsync(scratch, 0, ws.partials_off, s) != cudaSuccess) return LOOPVQ_ERR_CUDA;
-
-  DecodeParams p;
-  p.T = g.T; p.Tc = g.Tc; p.H = g.H; p.Hq = g.Hq; p.D = g.D; p.J = g.J; p.W = g.W; p.C = g.C;
-  p.loop_step = loop_step;
-  p.scale_log2 = softmax_scale * 1.4426950408889634f;
-  p.batch = layout->batch; p.n_sink = layout->n_sink; p.n_recent = layout->n_recent;
-  p.page = layout->page; p.max_ctx = layout->max_ctx_len;
-  p.ctx_len = layout->ctx_len; p.body_off = layout->body_off; p.win_off = layout->win_off;
-  p.body_pool_tokens = layout->body_pool_tokens; p.win_pool_tokens = layout->win_pool_tokens;
-  const size_t eb = cb_elem_bytes(g);
-  const size_t step_off = packed_slices_offset_bytes(g) + (size_t)loop_step * slice_elems_per_step(g) * eb;
-  p.cbK_slice = (const uint8_t*)cbK_packed + step_off;
-  p.cbV_slice = (const uint8_t*)cbV_packed + step_off;
-  const size_t blk_bytes = (size_t)g.H * layout->body_pool_tokens * g.J;
-  p.idxK = idxK_pool + (loop_step / g.Tc) * blk_bytes;
-  p.idxV = idxV_pool + (loop_step / g.Tc) * blk_bytes;
-  const size_t win_step = (size_t)g.H * layout->win_pool_tokens * g.D;
-  p.winK = (const __nv_bfloat16*)winK + loop_step * win_step;
-  p.winV = (const __nv_bfloat16*)winV + loop_step * win_step;
-  p.q = q; p.q_bf16 = q_dtype == LOOPVQ_BF16;
-  p.out = out; p.out_bf16 = out_dtype == LOOPVQ_BF16; p.lse = lse_out;
   p.status = fault_bits ? fault_bits : (uint32_t*)scratch;
   p.tickets = (uint32_t*)((uint8_t*)scratch + ws.tickets_off);
   p.partials = (float*)((uint8_t*)scratch + ws.partials_off);
-  p.split_len = pl.split_len;
-  p.max_splits = pl.max_splits;
-
-  p.static_inputs = (layout->flags & LOOPVQ_LAYOUT_STATIC_INPUTS) ? 1 : 0;
-  fill_layout_params(p, layout);
-
-  dim3 grid(g.Hq, pl.max_splits, layout->batch);
-#define LOOPVQ_LAUNCH(JJ, DD, CBT)                                                                    \
-  do {                                                                                               \
-    auto kfn = decode_kernel<JJ, DD, CBT>;                                                           \
-    if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, kDynSmem) != cudaSuccess) \
-      return LOOPVQ_ERR_CUDA;                                                                        \
-    if (launch_pdl((const void*)kfn, grid, s, &p) != cudaSuccess) return LOOPVQ_ERR_CUDA;           \
-    if (launch_pdl((const void*)merge_kernel<DD>, dim3(g.Hq, layout->batch), s, &p, DD, 0) !=          \
-        cudaSuccess)                                                                                 \
-      return LOOPVQ_ERR_CUDA;                                                                        \
-  } while (0)
-#define LOOPVQ_LAUNCH_J(DD, CBT)                      \
-  do {                                                \
-    if (g.J == 32) LOOPVQ_LAUNCH(32, DD, CBT);        \
-    else if (g.J == 16) LOOPVQ_LAUNCH(16, DD, CBT);   \
-    else LOOPVQ_LAUNCH(8, DD, CBT);                   \
-  } while (0)
-  if (g.D == 128) {
-    if (g.cb_bf16) LOOPVQ_LAUNCH_J(128, __nv_bfloat16);
-    else LOOPVQ_LAUNCH_J(128, float);
-  } else {
-    if (g.cb_bf16) LOOPVQ_LAUNCH_J(64, __nv_bfloat16);
-    else LOOPVQ_LAUNCH_J(64, float);
-  }
-#undef LOOPVQ_LAUNCH_J
-#undef LOOPVQ_LAUNCH
-  return cudaGetLastError() == cudaSuccess ? LOOPVQ_OK : LOOPVQ_ERR_CUDA;
+  return decode_launch(g, p, s);
 }

@@ -42,8 +42,9 @@ EXPORTED = [
     "loopvq_bits_per_element",
     "loopvq_codebook_packed_bytes", "loopvq_codebook_pack", "loopvq_index_pool_bytes",
     "loopvq_index_pool_pack", "loopvq_index_pool_unpack", "loopvq_encode", "loopvq_read_encode_faults",
-    "loopvq_codebook_update_workspace_bytes", "loopvq_codebook_update",
+    "loopvq_codebook_update_workspace_bytes", "loopvq_codebook_update", "loopvq_codebook_grad",
     "loopvq_decode_workspace_bytes", "loopvq_decode_attn", "loopvq_decode_attn_noalloc",
+    "loopvq_decode_steps_workspace_bytes", "loopvq_decode_attn_steps",
     "loopvq_read_device_status",
     "loopvq_clear_device_status", "loopvq_dense_decode_workspace_bytes", "loopvq_dense_decode_attn",
 ]
@@ -96,9 +97,14 @@ def _load() -> ctypes.CDLL:
         "loopvq_codebook_update_workspace_bytes": (SZ, [D]),
         "loopvq_codebook_update": (ctypes.c_int, [D, ctypes.c_int, P, ctypes.c_int, I64, I64, I64, I64, U8P, I64, I64,
                                                   P, P, P, P, SZ, P]),
+        "loopvq_codebook_grad": (ctypes.c_int, [D, P, P, L, U8P, U8P, P, ctypes.c_int, I32, F, P, P, P, F, P, P,
+                                                P, P, P]),
         "loopvq_decode_workspace_bytes": (SZ, [D, L]),
         "loopvq_decode_attn": (ctypes.c_int, [D, P, P, L, U8P, U8P, P, P, P, ctypes.c_int, I32, F, P,
                                               ctypes.c_int, P, P, SZ, P]),
+        "loopvq_decode_steps_workspace_bytes": (SZ, [D, L, I32]),
+        "loopvq_decode_attn_steps": (ctypes.c_int, [D, P, P, L, U8P, U8P, P, P, P, ctypes.c_int, I32, I32, F, P,
+                                                    ctypes.c_int, P, P, SZ, P]),
         "loopvq_decode_attn_noalloc": (ctypes.c_int, [D, P, P, L, U8P, U8P, P, P, P, ctypes.c_int, I32, F, P,
                                                       ctypes.c_int, P, P, P]),
         "loopvq_read_device_status": (ctypes.c_int, [P, ctypes.POINTER(ctypes.c_uint32), P]),
@@ -167,10 +173,13 @@ def make_desc(n_loop, tc, n_heads_kv, head_dim, group_elems, n_codes=256, n_head
 def make_layout(batch, n_sink, n_recent, page, max_ctx_len, ctx_len, body_off, win_off,
                 body_pool_tokens, win_pool_tokens, flags=0, body_pages=None, body_page_tokens=0,
                 max_body_pages=0, win_head=None, win_ring=0, new_k=None, new_v=None) -> loopvq_cache_layout:
-    return loopvq_cache_layout(batch, n_sink, n_recent, page, max_ctx_len, flags, _ptr(ctx_len), _ptr(body_off),
-                               _ptr(win_off), body_pool_tokens, win_pool_tokens, _ptr(body_pages),
-                               body_page_tokens, max_body_pages, _ptr(win_head), win_ring, 0, _ptr(new_k),
-                               _ptr(new_v))
+    lay = loopvq_cache_layout(batch, n_sink, n_recent, page, max_ctx_len, flags, _ptr(ctx_len), _ptr(body_off),
+                              _ptr(win_off), body_pool_tokens, win_pool_tokens, _ptr(body_pages),
+                              body_page_tokens, max_body_pages, _ptr(win_head), win_ring, 0, _ptr(new_k),
+                              _ptr(new_v))
+    # the struct holds raw device pointers: keep the arrays alive with it
+    lay._keep = (ctx_len, body_off, win_off, body_pages, win_head, new_k, new_v)
+    return lay
 
 
 # ------------------------------------------------------------------ entry points
@@ -253,6 +262,17 @@ def loopvq_codebook_update(desc, kind, x, n_tokens, stride_t, stride_n, stride_h
         _ptr(workspace), _nbytes(workspace), _stream(stream)))
 
 
+def loopvq_codebook_grad(desc, cbK, cbV, layout, idxK_pool, idxV_pool, q, loop_step, softmax_scale, out, lse,
+                         target, weight, gradK, gradV, loss_out=None, fault_bits=None, stream=None) -> None:
+    """Adds the codebook gradients of weight * sum ||out - target||^2 at loop
+    step ``loop_step`` to ``gradK``/``gradV`` (canonical fp32) and the loss to
+    ``loss_out`` (one-element fp32 tensor, optional)."""
+    _check("loopvq_codebook_grad", _lib.loopvq_codebook_grad(
+        ctypes.byref(desc), _ptr(cbK), _ptr(cbV), ctypes.byref(layout), _ptr(idxK_pool), _ptr(idxV_pool), _ptr(q),
+        _dtype_code(q), loop_step, softmax_scale, _ptr(out), _ptr(lse), _ptr(target), weight, _ptr(gradK),
+        _ptr(gradV), _ptr(loss_out), _ptr(fault_bits), _stream(stream)))
+
+
 def loopvq_decode_workspace_bytes(desc, layout) -> int:
     return _lib.loopvq_decode_workspace_bytes(ctypes.byref(desc), ctypes.byref(layout))
 
@@ -265,6 +285,20 @@ def loopvq_decode_attn(desc, cbK_packed, cbV_packed, layout, idxK_pool, idxV_poo
         ctypes.byref(desc), _ptr(cbK_packed), _ptr(cbV_packed), ctypes.byref(layout), _ptr(idxK_pool),
         _ptr(idxV_pool), _ptr(winK), _ptr(winV), _ptr(q), _dtype_code(q), loop_step, softmax_scale,
         _ptr(out), _dtype_code(out), _ptr(lse_out), _ptr(workspace), wb, _stream(stream)))
+
+
+def loopvq_decode_steps_workspace_bytes(desc, layout, n_steps) -> int:
+    return _lib.loopvq_decode_steps_workspace_bytes(ctypes.byref(desc), ctypes.byref(layout), n_steps)
+
+
+def loopvq_decode_attn_steps(desc, cbK_packed, cbV_packed, layout, idxK_pool, idxV_pool, winK, winV, q,
+                             first_step, n_steps, softmax_scale, out, lse_out, workspace, stream=None) -> None:
+    """Loop steps first_step .. first_step+n_steps-1 in one launch; q, out
+    and lse_out carry a leading [n_steps] axis."""
+    _check("loopvq_decode_attn_steps", _lib.loopvq_decode_attn_steps(
+        ctypes.byref(desc), _ptr(cbK_packed), _ptr(cbV_packed), ctypes.byref(layout), _ptr(idxK_pool),
+        _ptr(idxV_pool), _ptr(winK), _ptr(winV), _ptr(q), _dtype_code(q), first_step, n_steps, softmax_scale,
+        _ptr(out), _dtype_code(out), _ptr(lse_out), _ptr(workspace), _nbytes(workspace), _stream(stream)))
 
 
 def prepare_decode_attn(desc, cbK_packed, cbV_packed, layout, idxK_pool, idxV_pool, winK, winV, q, loop_step,

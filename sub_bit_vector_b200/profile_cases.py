@@ -9,6 +9,10 @@ holds well under 2 GB on the device:
                 steps, Tc = 4, G = 16 (0.5 bit): one decode launch per loop
                 step (4 launches).
 - ``decode-q``: the same at G = 32 (0.25 bit).
+- ``decode-gqa``: the same context with 8 KV heads and 16 query heads
+                (GQA ratio 2), 4 launches.
+- ``decode-steps``: the ``decode`` case as one launch of all 4 loop steps
+                (loopvq_decode_attn_steps), 2 launches.
 - ``encode``  : loop-axis encode of a [4][32768][16][128] bf16 tensor at
                 Tc = 4, G = 16 (tensor-core kernel), 2 launches.
 - ``encode-f32``: the same tensor in fp32 (CUDA-core kernel), 2 launches.
@@ -37,6 +41,40 @@ def _decode(G):
         c.decode(t)
     torch.cuda.synchronize()
     print("decode status", c.device_status(), "algorithmic bytes per launch", c.algorithmic_bytes())
+
+
+def _decode_gqa():
+    c = cache.DecodeCache(n_loop=4, tc=4, n_heads_kv=8, head_dim=128, group_elems=16, ctx_lens=[32768], n_heads_q=16)
+    cb = synth.uniform_codebook(1, 1, 8, 32, 256, 4, 4)
+    c.set_codebooks(cb, cb)
+    c.idxK.copy_(synth.device_codes(2, c.idxK.numel()))
+    c.idxV.copy_(synth.device_codes(3, c.idxV.numel()))
+    c.winK.normal_()
+    c.winV.normal_()
+    c.q.normal_()
+    for t in range(4):
+        c.decode(t)
+    torch.cuda.synchronize()
+    print("decode-gqa status", c.device_status(), "algorithmic bytes per launch", c.algorithmic_bytes())
+
+
+def _decode_steps():
+    c = cache.DecodeCache(n_loop=4, tc=4, n_heads_kv=16, head_dim=128, group_elems=16, ctx_lens=[32768])
+    cb = synth.uniform_codebook(1, 1, 16, 32, 256, 4, 4)
+    c.set_codebooks(cb, cb)
+    c.idxK.copy_(synth.device_codes(2, c.idxK.numel()))
+    c.idxV.copy_(synth.device_codes(3, c.idxV.numel()))
+    c.winK.normal_()
+    c.winV.normal_()
+    q = synth.device_normal(4, (4, 1, 16, 128)).to(torch.bfloat16)
+    out = torch.zeros((4, 1, 16, 128), dtype=torch.float32, device="cuda")
+    lse = torch.zeros((4, 1, 16), dtype=torch.float32, device="cuda")
+    ws = torch.zeros(L.loopvq_decode_steps_workspace_bytes(c.desc, c.layout, 4), dtype=torch.uint8, device="cuda")
+    for _ in range(2):
+        L.loopvq_decode_attn_steps(c.desc, c.cbK, c.cbV, c.layout, c.idxK, c.idxV, c.winK, c.winV, q, 0, 4,
+                                   128 ** -0.5, out, lse, ws)
+    torch.cuda.synchronize()
+    print("decode-steps status", L.loopvq_read_device_status(ws))
 
 
 def _encode(dtype):
@@ -75,6 +113,8 @@ def _page():
 CASES = {
     "decode": lambda: _decode(16),
     "decode-q": lambda: _decode(32),
+    "decode-gqa": _decode_gqa,
+    "decode-steps": _decode_steps,
     "encode": lambda: _encode(torch.bfloat16),
     "encode-f32": lambda: _encode(torch.float32),
     "page": _page,

@@ -161,3 +161,49 @@ def test_paged_ring_and_new_token_layout_validation():
     assert L.loopvq_decode_workspace_bytes(d, _layout(new_k=FAKE, new_v=FAKE)) > 0
     assert L.loopvq_decode_workspace_bytes(d, _layout(new_k=FAKE)) == 0                         # K without V
     assert L.loopvq_decode_workspace_bytes(d, _layout(new_k=FAKE + 2, new_v=FAKE)) == 0         # misaligned
+
+
+def test_codebook_grad_rejects_bad_arguments_before_launch():
+    import ctypes
+    d = L.make_desc(4, 4, 16, 128, 16)
+    lay = _layout()
+    D, Lp = ctypes.byref(d), ctypes.byref(lay)
+    fn = L._lib.loopvq_codebook_grad
+
+    def call(desc=D, layout=Lp, idxK=FAKE, q=FAKE, qd=L.LOOPVQ_BF16, t=0, lse=FAKE, target=FAKE, gk=FAKE,
+             weight=1.0):
+        return fn(desc, FAKE, FAKE, layout, idxK, FAKE, q, qd, t, 0.088, FAKE, lse, target, weight, gk, FAKE, None,
+                  None, None)
+    assert call(t=4) == L.LOOPVQ_ERR_INVALID_ARG
+    assert call(t=-1) == L.LOOPVQ_ERR_INVALID_ARG
+    assert call(idxK=FAKE + 8) == L.LOOPVQ_ERR_INVALID_ARG
+    assert call(q=None) == L.LOOPVQ_ERR_INVALID_ARG
+    assert call(lse=None) == L.LOOPVQ_ERR_INVALID_ARG
+    assert call(target=None) == L.LOOPVQ_ERR_INVALID_ARG
+    assert call(gk=None) == L.LOOPVQ_ERR_INVALID_ARG
+    assert call(qd=7) == L.LOOPVQ_ERR_INVALID_ARG
+    assert call(weight=float("nan")) == L.LOOPVQ_ERR_INVALID_ARG
+    bad = L.make_desc(4, 4, 16, 128, 8)     # J = 64
+    assert call(desc=ctypes.byref(bad)) == L.LOOPVQ_ERR_UNSUPPORTED
+    lay2 = _layout(ctx_len=None)
+    assert call(layout=ctypes.byref(lay2)) == L.LOOPVQ_ERR_INVALID_ARG
+
+
+def test_decode_steps_rejects_bad_step_ranges():
+    import ctypes
+    d = L.make_desc(4, 2, 16, 128, 8)
+    lay = _layout()
+    D, Lp = ctypes.byref(d), ctypes.byref(lay)
+    assert L._lib.loopvq_decode_steps_workspace_bytes(D, Lp, 4) > L._lib.loopvq_decode_steps_workspace_bytes(D, Lp, 1)
+    assert L._lib.loopvq_decode_steps_workspace_bytes(D, Lp, 1) == L._lib.loopvq_decode_workspace_bytes(D, Lp)
+    assert L._lib.loopvq_decode_steps_workspace_bytes(D, Lp, 5) == 0
+    assert L._lib.loopvq_decode_steps_workspace_bytes(D, Lp, 0) == 0
+    fn = L._lib.loopvq_decode_attn_steps
+
+    def call(first, n, wsb=1 << 30):
+        return fn(D, FAKE, FAKE, Lp, FAKE, FAKE, FAKE, FAKE, FAKE, L.LOOPVQ_BF16, first, n, 0.088, FAKE, L.LOOPVQ_F32,
+                  None, FAKE, wsb, None)
+    assert call(0, 0) == L.LOOPVQ_ERR_INVALID_ARG
+    assert call(2, 3) == L.LOOPVQ_ERR_INVALID_ARG
+    assert call(-1, 2) == L.LOOPVQ_ERR_INVALID_ARG
+    assert call(1, 2, wsb=256) == L.LOOPVQ_ERR_WORKSPACE_TOO_SMALL
