@@ -24,8 +24,8 @@
 //   Every split writes its (m, l, o); a small merge kernel, launched right
 //   after as a programmatic dependent, combines them by log-sum-exp.
 //
-// Fixed-point bound: a split holds n <= kSplitCap < 2^12 tokens and S is
-// chosen so that n * 2^S < 2^32, so no bin or sum can overflow.
+// Fixed-point bound: a split holds n <= 8192 = 2^13 tokens and S = clz(n),
+// so n * (2^S + 1) < 2^32: no bin or sum can overflow.
 
 #include <math.h>
 #include <stdio.h>
@@ -38,12 +38,24 @@ namespace loopvq {
 
 constexpr int kNW = 16;                      // consumer warps
 constexpr int kThreads = (kNW + 1) * 32;     // + one producer warp
-constexpr int kStages = 4;
-// With static inputs, chunks a body CTA streams before the previous kernel
-// has finished (the rest follow the dependency).
-constexpr int kPreWaitChunks = 4;
 constexpr int kStageBytes = 32768;
-constexpr int kSplitCap = 4064;              // max body tokens per split, multiple of 32
+// Ring depth and split cap.  The default is a 4-stage ring and splits of up
+// to 4064 tokens (a 16 KB score buffer).  With 16 slots and a value slice of
+// at most two stages (bf16 at D = 128, any at D = 64) the ring drops to three
+// stages and the cap doubles to 8192 tokens (a 32 KB score buffer), so a 64K
+// context needs 8 splits per head instead of 17 and fits one wave on 148 SMs.
+// With static inputs a CTA streams its first ring-full of chunks before the
+// previous kernel has finished; the producer waits for that kernel before it
+// waits for a stage to drain (the consumers only start after it).
+constexpr int kSplitCap = 4064;              // default max body tokens per split, multiple of 32
+constexpr int kSplitCapLong = 8192;
+constexpr bool long_splits(int J, int D, int cb_bytes) { return J == 16 && 256 * D * cb_bytes <= 2 * kStageBytes; }
+template <int J, int D, typename CBT>
+struct Ring {
+  static constexpr bool kLong = long_splits(J, D, (int)sizeof(CBT));
+  static constexpr int kStages = kLong ? 3 : 4;
+  static constexpr int kCap = kLong ? kSplitCapLong : kSplitCap;
+};
 // One 64 KB region of 256 rows (one per code) of 64 four-byte columns holds
 // the lookup table during pass K and the histogram during pass V.  Column x
 // stands for slot x mod J (the table is replicated 64/J times), so lane l at
@@ -53,7 +65,6 @@ constexpr int kSplitCap = 4064;              // max body tokens per split, multi
 // bytes 2-3) and the step's 4*s is the load's immediate offset.
 constexpr int kRegionBytes = 65536;
 constexpr int kCols = 64;
-constexpr int kScoresBytes = kSplitCap * 4;
 constexpr int kMiscBytes = 4096;
 // allocation: the region, the ring, scores and misc, plus room to align the
 // region to 64 KB (the part below the region holds misc, scores and ring
@@ -89,7 +100,7 @@ struct DecodeParams {
   // pools by a code block's.
   int n_steps;
   int64_t slice_step_elems, win_step_elems, idx_blk_bytes;
-  int split_len;   // body tokens per split (multiple of 32, <= kSplitCap)
+  int split_len;   // body tokens per split (multiple of 32, <= the kernel's cap)
   int max_splits;  // grid.x
   int static_inputs;  // layout arrays, index pools and codebooks are not being written by earlier kernels
   int static_windows;  // nor the window pools
@@ -297,6 +308,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
   const int h = hq / group;
   constexpr int W = D / J;
   constexpr int kPer = 256 * J / (kNW * 32);   // lookup-table entries per consumer thread
+  constexpr int kStages = Ring<J, D, CBT>::kStages;
+  constexpr int kScoresBytes = Ring<J, D, CBT>::kCap * 4;
 
   griddep_launch_dependents();
   if (!p.static_inputs) griddep_wait();
@@ -418,7 +431,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
     int pbase = -1 << 30, pcache = -1;  // page ids pbase + lane
     for (int k = 0; k < n_chunks + n_slice; ++k) {
       const int s = k % kStages;
-      if (k == kPreWaitChunks && p.static_inputs && !is_window) griddep_wait();
+      if (k == kStages && p.static_inputs) griddep_wait();
       if (k >= kStages) {
         int ok = 1;
         if (leader) ok = mbar_wait_bounded(smem_u32(empty_bar + s), ((k / kStages) - 1) & 1) ? 1 : 0;
@@ -907,9 +920,9 @@ static cudaError_t launch_pdl(const void* fn, dim3 grid, cudaStream_t s, DecodeP
 struct DecodePlan {
   int n_body_splits, split_len, max_splits;
 };
-inline DecodePlan decode_plan(int64_t units, int max_body, int n_sm) {
+inline DecodePlan decode_plan(int64_t units, int max_body, int n_sm, int cap = kSplitCap) {
   DecodePlan pl;
-  int need = (max_body + kSplitCap - 1) / kSplitCap;  // fixed-point bound
+  int need = (max_body + cap - 1) / cap;  // score buffer and fixed-point bound
   int fill = (int)(n_sm / (units > 0 ? units : 1)) - 1;  // one window split per unit
   int cap_by_tiles = (max_body + 255) / 256;             // >= 256 tokens per split
   int s = need;
@@ -918,7 +931,7 @@ inline DecodePlan decode_plan(int64_t units, int max_body, int n_sm) {
   int len = (max_body + s - 1) / s;
   len = ((len + 31) / 32) * 32;
   if (len < 32) len = 32;
-  if (len > kSplitCap) len = kSplitCap;
+  if (len > cap) len = cap;
   pl.split_len = len;
   pl.n_body_splits = max_body > 0 ? (max_body + len - 1) / len : 0;
   pl.max_splits = pl.n_body_splits + 1;
@@ -1004,7 +1017,8 @@ static loopvq_status decode_setup(const loopvq_codebook_desc* desc, const void* 
       ((uintptr_t)winV & 15) || ((uintptr_t)cbK_packed & 15) || ((uintptr_t)cbV_packed & 15))
     return LOOPVQ_ERR_INVALID_ARG;
   const int64_t units = (int64_t)layout->batch * g.Hq * n_steps;
-  const DecodePlan pl = decode_plan(units, max_body_tokens(layout), device_sm_count());
+  const int cap = long_splits(g.J, g.D, (int)cb_elem_bytes(g)) ? kSplitCapLong : kSplitCap;
+  const DecodePlan pl = decode_plan(units, max_body_tokens(layout), device_sm_count(), cap);
   if (units > 65535LL * 65535LL || pl.max_splits > kMaxCombineSplits || layout->batch > 65535 ||
       (int64_t)g.Hq * n_steps > 65535)
     return LOOPVQ_ERR_UNSUPPORTED;
