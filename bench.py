@@ -375,14 +375,15 @@ def all_steps_measurement(layers, device, reps=400):
         with torch.cuda.graph(g, stream=s):
             launch(b)
         graphs.append(g)
-    for i in range(2 * len(graphs)):
-        graphs[i % len(graphs)].replay()
-    torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(s)
-    for i in range(reps):
-        graphs[i % len(graphs)].replay()
-    e1.record(s)
+    with torch.cuda.stream(s):   # replay() launches on the current stream
+        for i in range(2 * len(graphs)):
+            graphs[i % len(graphs)].replay()
+        torch.cuda.synchronize()
+        e0.record(s)
+        for i in range(reps):
+            graphs[i % len(graphs)].replay()
+        e1.record(s)
     torch.cuda.synchronize()
     us_launch = e0.elapsed_time(e1) * 1e3 / reps
     faults = max(L.loopvq_read_device_status(b[4])[1] for b in bufs)

@@ -39,20 +39,21 @@ namespace loopvq {
 constexpr int kNW = 16;                      // consumer warps
 constexpr int kThreads = (kNW + 1) * 32;     // + one producer warp
 constexpr int kStageBytes = 32768;
-// Ring depth and split cap.  The default is a 4-stage ring and splits of up
-// to 4064 tokens (a 16 KB score buffer).  With 16 slots and a value slice of
-// at most two stages (bf16 at D = 128, any at D = 64) the ring drops to three
-// stages and the cap doubles to 8192 tokens (a 32 KB score buffer), so a 64K
-// context needs 8 splits per head instead of 17 and fits one wave on 148 SMs.
+// Ring depth and split cap.  When the value slice fits two stages (bf16 at
+// D = 128, either type at D = 64) the ring has three stages and splits of up
+// to 8192 tokens (a 32 KB score buffer): a 64K context needs 8 splits per
+// head instead of 17 and fits one wave on 148 SMs, and long batched contexts
+// pay the per-split start-up and epilogue half as often.  An fp32 slice at
+// D = 128 takes four stages, which leaves 16 KB of scores: 4064 tokens.
 // With static inputs a CTA streams its first ring-full of chunks before the
 // previous kernel has finished; the producer waits for that kernel before it
 // waits for a stage to drain (the consumers only start after it).
 constexpr int kSplitCap = 4064;              // default max body tokens per split, multiple of 32
 constexpr int kSplitCapLong = 8192;
-constexpr bool long_splits(int J, int D, int cb_bytes) { return J == 16 && 256 * D * cb_bytes <= 2 * kStageBytes; }
+constexpr bool long_splits(int D, int cb_bytes) { return 256 * D * cb_bytes <= 2 * kStageBytes; }
 template <int J, int D, typename CBT>
 struct Ring {
-  static constexpr bool kLong = long_splits(J, D, (int)sizeof(CBT));
+  static constexpr bool kLong = long_splits(D, (int)sizeof(CBT));
   static constexpr int kStages = kLong ? 3 : 4;
   static constexpr int kCap = kLong ? kSplitCapLong : kSplitCap;
 };
@@ -1017,7 +1018,7 @@ static loopvq_status decode_setup(const loopvq_codebook_desc* desc, const void* 
       ((uintptr_t)winV & 15) || ((uintptr_t)cbK_packed & 15) || ((uintptr_t)cbV_packed & 15))
     return LOOPVQ_ERR_INVALID_ARG;
   const int64_t units = (int64_t)layout->batch * g.Hq * n_steps;
-  const int cap = long_splits(g.J, g.D, (int)cb_elem_bytes(g)) ? kSplitCapLong : kSplitCap;
+  const int cap = long_splits(g.D, (int)cb_elem_bytes(g)) ? kSplitCapLong : kSplitCap;
   const DecodePlan pl = decode_plan(units, max_body_tokens(layout), device_sm_count(), cap);
   if (units > 65535LL * 65535LL || pl.max_splits > kMaxCombineSplits || layout->batch > 65535 ||
       (int64_t)g.Hq * n_steps > 65535)
