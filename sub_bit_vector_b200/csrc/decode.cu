@@ -380,9 +380,17 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
   };
   const uint32_t misc_a = place(kMiscBytes);
   const uint32_t sc_a = place(kScoresBytes);
+  // The three-stage ring is one block (stage i at ring_a + i * kStageBytes);
+  // the four-stage ring puts one stage below the region.
   uint32_t stage_a[kStages];
+  if constexpr (Ring<J, D, CBT>::kLong) {
+    const uint32_t ring_a = place(kStages * kStageBytes);
 #pragma unroll
-  for (int i = 0; i < kStages; ++i) stage_a[i] = place(kStageBytes);
+    for (int i = 0; i < kStages; ++i) stage_a[i] = ring_a + i * kStageBytes;
+  } else {
+#pragma unroll
+    for (int i = 0; i < kStages; ++i) stage_a[i] = place(kStageBytes);
+  }
   if (hi > sbase + kDynSmem) {  // cannot happen with the 1 KB reserved window start
     if (tid == 0) set_fault(p.status, LOOPVQ_FAULT_TIMEOUT);
     return;
@@ -390,7 +398,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
   uint8_t* const region_p = dyn + (region - sbase);
   float* const lut = reinterpret_cast<float*>(region_p);         // pass K: lut[c*64 + col]
   uint32_t* const hist = reinterpret_cast<uint32_t*>(region_p);  // pass V: hist[c*64 + col]
-  auto stage_ptr = [&](int i) -> uint8_t* { return dyn + (stage_a[i] - sbase); };
+  auto stage_ptr = [&](int i) -> uint8_t* {
+    if constexpr (Ring<J, D, CBT>::kLong) return dyn + (stage_a[0] - sbase) + i * kStageBytes;
+    else return dyn + (stage_a[i] - sbase);
+  };
   float* const sc = reinterpret_cast<float*>(dyn + (sc_a - sbase));
   uint8_t* const misc = dyn + (misc_a - sbase);
   uint64_t* const full_bar = reinterpret_cast<uint64_t*>(misc);
@@ -441,7 +452,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
           break;
         }
       }
-      const uint32_t dst = stage_a[s];
+      const uint32_t dst = Ring<J, D, CBT>::kLong ? stage_a[0] + (uint32_t)s * kStageBytes : stage_a[s];
       const uint32_t fb = smem_u32(full_bar + s);
       if (k >= n_chunks) {  // a piece of the value codebook slice, for the epilogue
         const uint32_t off = (uint32_t)(k - n_chunks) * kStageBytes;
