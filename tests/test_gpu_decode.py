@@ -344,3 +344,19 @@ def test_host_argument_errors_on_gpu():
         L.loopvq_decode_attn(c.desc, c.cbK, c.cbV, c.layout, c.idxK[1:], c.idxV, c.winK, c.winV, c.q, 0, 0.1,
                              c.out, c.lse, c.workspace)
     assert e.value.status == L.LOOPVQ_ERR_INVALID_ARG
+
+
+def test_long_split_boundaries():
+    """Three-stage ring (bf16 codebooks, D = 128): 16 heads x 10 requests
+    leave no room to fill SMs, so the planner cuts 8192-token splits; bodies
+    just below, at and above one and two split lengths."""
+    ctx = [320 + 16384, 320 + 8192 - 8, 320 + 8192, 320 + 8192 + 8, 320 + 16384 - 8, 330, 3000, 12000, 321, 700]
+    case = Case(seed=11, ctx_lens=ctx, H=16, keep=[0, 1, 2, 3, 4])
+    for t in (0, 3):
+        case.check(t)
+
+
+def test_gqa_ratio_four():
+    case = Case(seed=12, ctx_lens=[5000, 333, 1], H=2, Hq=8)
+    for t in (1, 2):
+        case.check(t)

@@ -231,3 +231,108 @@ def test_fine_tuning_loop_lowers_attention_error_at_every_step():
         loss, grads = losses_and_grads(cb)
     assert np.all(loss <= 0.85 * first), (first, loss)
     assert L.loopvq_read_device_status(ws)[1] == 0
+
+
+def test_codebook_grad_paged_layout_matches_contiguous():
+    """The same logical cache with the body in shuffled 256-token pages gives
+    the same gradients (up to the order of the float atomics)."""
+    L = _L()
+    T, tc, G, D = 4, 4, 16, 128
+    ctx = [3000, 700, 333]
+    dc, cbk, cbv, cbk_d, cbv_d, codes, wins = _cache_case(tc, G, D, ctx, torch.bfloat16, Hq=2, H=2, seed=500)
+    bpt = 256
+    max_pages = -(-max(dc.splits[r][1] for r in range(len(ctx))) // bpt)
+    n_phys = len(ctx) * max_pages + 2
+    rng = np.random.default_rng(501)
+    perm = rng.permutation(n_phys)
+    pool_tokens = n_phys * bpt
+    idxK = torch.zeros(L.loopvq_index_pool_bytes(dc.desc, pool_tokens), dtype=torch.uint8, device="cuda")
+    idxV = torch.zeros_like(idxK)
+    pages = np.full((len(ctx), max_pages), -1, dtype=np.int32)
+    nxt = 0
+    for r in range(len(ctx)):
+        body = dc.splits[r][1]
+        ck, cv = codes[r]
+        for pi in range(-(-body // bpt)):
+            pages[r, pi] = perm[nxt]
+            nxt += 1
+            n = min(bpt, body - pi * bpt)
+            for kind, src, pool in ((0, ck, idxK), (1, cv, idxV)):
+                t = torch.from_numpy(np.ascontiguousarray(src[:, :, pi * bpt:pi * bpt + n])).cuda()
+                L.loopvq_index_pool_pack(dc.desc, kind, t, n, pool, int(pages[r, pi]) * bpt, pool_tokens)
+    pages_dev = torch.from_numpy(pages).cuda()
+    lay = L.make_layout(len(ctx), dc.n_sink, dc.n_recent, dc.page, dc.max_ctx_len, dc.ctx_dev, dc.body_off_dev,
+                        dc.win_off_dev, pool_tokens, dc.win_pool_tokens, L.LOOPVQ_LAYOUT_PAGED_BODY, pages_dev, bpt,
+                        max_pages)
+    t, scale = 2, D ** -0.5
+    q = synth.round_bf16(rng.standard_normal((len(ctx), 2, D)).astype(np.float32))
+    dc.set_queries(q)
+    dc.decode(t, scale)
+    tgt = torch.from_numpy((0.05 * rng.standard_normal((len(ctx), 2, D))).astype(np.float32)).cuda()
+    grads = []
+    for layout, ik, iv in ((dc.layout, dc.idxK, dc.idxV), (lay, idxK, idxV)):
+        gk = torch.zeros(cbk.shape, dtype=torch.float32, device="cuda")
+        gv = torch.zeros_like(gk)
+        faults = torch.zeros(1, dtype=torch.int32, device="cuda")
+        L.loopvq_codebook_grad(dc.desc, cbk_d, cbv_d, layout, ik, iv, dc.q, t, scale, dc.out, dc.lse, tgt, 1.0, gk, gv,
+                               None, faults)
+        torch.cuda.synchronize()
+        assert int(faults.item()) == 0
+        grads.append((gk.cpu().numpy(), gv.cpu().numpy()))
+    assert _normwise(grads[1][0], grads[0][0]) <= 1e-5
+    assert _normwise(grads[1][1], grads[0][1]) <= 1e-5
+    assert np.any(grads[0][0] != 0)
+
+
+def test_codebook_grad_code_out_of_range_sets_fault_and_skips_token():
+    """n_codes = 100: a stored code >= 100 raises the code-range bit and its
+    token adds nothing; the rest still matches the oracle without it."""
+    L = _L()
+    C = _cache()
+    T, tc, H, D, G, n_codes = 4, 4, 1, 64, 16, 100
+    dc = C.DecodeCache(n_loop=T, tc=tc, n_heads_kv=H, head_dim=D, group_elems=G, ctx_lens=[1200], n_codes=n_codes,
+                       cb_dtype=torch.float32, q_dtype=torch.float32)
+    W = G // tc
+    J = D // W
+    cbk = synth.uniform_codebook(600, 1, H, J, n_codes, tc, W, bf16=False)
+    cbv = synth.uniform_codebook(601, 1, H, J, n_codes, tc, W, bf16=False)
+    dc.set_codebooks(cbk, cbv)
+    s, body, rec = dc.splits[0]
+    ck = synth.random_codes(602, 1, H, body, J, n_codes)
+    cv = synth.random_codes(603, 1, H, body, J, n_codes)
+    rng = np.random.default_rng(604)
+    wk = rng.standard_normal((T, H, s + rec, D)).astype(np.float32)
+    wv = rng.standard_normal((T, H, s + rec, D)).astype(np.float32)
+    dc.set_request_window(0, wk, wv)
+    dc.set_request_codes(0, ck, cv)
+    t, scale = 1, D ** -0.5
+    q = rng.standard_normal((1, H, D)).astype(np.float32)
+    dc.set_queries(q)
+    dc.decode(t, scale)                          # forward with valid codes
+    bad = ck.copy()
+    bad[0, 0, 77, 5] = 200                       # token 77's key code out of range
+    dc.set_request_codes(0, bad, cv)
+    target = (0.05 * rng.standard_normal((1, H, D))).astype(np.float32)
+    gk = torch.zeros(cbk.shape, dtype=torch.float32, device="cuda")
+    gv = torch.zeros_like(gk)
+    faults = torch.zeros(1, dtype=torch.int32, device="cuda")
+    L.loopvq_codebook_grad(dc.desc, torch.from_numpy(cbk).cuda(), torch.from_numpy(cbv).cuda(), dc.layout, dc.idxK,
+                           dc.idxV, dc.q, t, scale, dc.out, dc.lse, torch.from_numpy(target).cuda(), 1.0, gk, gv, None,
+                           faults)
+    torch.cuda.synchronize()
+    assert int(faults.item()) & L.LOOPVQ_FAULT_CODE_RANGE
+    # oracle over the valid codes; token 77 is skipped on the GPU, so compare
+    # every entry that token 77 does not touch (its K and V codeword per slot)
+    _, ref_k, ref_v, _ = O.attention_mse_codebook_grad(q[0], t, tc, ck, cv, cbk, cbv, wk[t], wv[t], scale, target[0])
+    got_k = gk.cpu().numpy().astype(np.float64)
+    got_v = gv.cpu().numpy().astype(np.float64)
+    mk = np.ones(got_k.shape, dtype=bool)
+    mv = np.ones(got_v.shape, dtype=bool)
+    for j in range(J):
+        mk[0, 0, j, ck[0, 0, 77, j]] = False
+        mv[0, 0, j, cv[0, 0, 77, j]] = False
+    scale_k = np.max(np.abs(ref_k))
+    scale_v = np.max(np.abs(ref_v))
+    assert np.max(np.abs(got_k[mk] - ref_k[mk])) <= 2e-3 * scale_k
+    assert np.max(np.abs(got_v[mv] - ref_v[mv])) <= 2e-3 * scale_v
+    assert np.all(np.isfinite(got_k)) and np.all(np.isfinite(got_v))
