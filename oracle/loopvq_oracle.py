@@ -65,6 +65,12 @@ __all__ = [
     "kmeans",
     "distortion",
     "attention_mse_codebook_grad",
+    "quantize4_group",
+    "dequantize4",
+    "residual_encode",
+    "residual_reconstruct",
+    "residual_decode_attention",
+    "residual_bits_per_element",
 ]
 
 
@@ -482,3 +488,143 @@ def attention_mse_codebook_grad(q, loop_step, tc, idx_k, idx_v, codebook_k, code
             np.add.at(grad_k[b, h, j, :, tt, :], ck, np.outer(ds_body, scale * q[hq, sl]))
             np.add.at(grad_v[b, h, j, :, tt, :], cv, np.outer(p_body, g[sl]))
     return loss, grad_k, grad_v, out
+
+
+# --------------------------------------------------------------------------
+# second workload: adjacent-loop KV-residual quantization (4-bit)
+# --------------------------------------------------------------------------
+# FlashLoop page (thelatestinai.com, "Figure 2 (c)", "Figure 3 (c-d)", "Table
+# 2", "Figure 4"): K/V residuals between adjacent loop steps shrink with loop
+# depth, and recursively quantizing adjacent-loop residuals gives a lower
+# reconstruction error than quantizing every loop's complete K/V; the method
+# uses 4-bit residuals along the axes of per-loop KIVI4.  Readings where the
+# page is silent: KIVI's quantizer (asymmetric, 16 levels, min and scale per
+# group of 32; keys grouped per channel over 32 consecutive tokens, values
+# per token over 32 consecutive channels; min and scale stored in fp16);
+# step 0 codes K_0 itself and step t codes R_t = K_t - Khat_{t-1}, the
+# residual against the previous step's reconstruction, so that Khat_t =
+# Khat_{t-1} + Q(R_t) and errors do not pile up.  Every quantization decision
+# is taken in fp32 with separately rounded operations (the kernel's
+# precision), so codes and parameters are exact.
+
+RESIDUAL_GROUP = 32
+
+
+def quantize4_group(x):
+    """4-bit asymmetric quantization of one group (KIVI's quantizer).
+
+    lo = min x, scale = (max x - lo) / 15 in fp32; both are stored in fp16
+    (round to nearest even); code = clamp(rint((x - lo_h) / scale_h), 0, 15)
+    with fp32 subtraction and division, or 0 when scale_h is 0.  Returns
+    ``(codes uint8, lo_h, scale_h)`` (the last two as np.float16).
+    """
+    x = np.asarray(x, dtype=np.float32)
+    lo = np.min(x)
+    hi = np.max(x)
+    scale = np.float32(np.float32(hi - lo) / np.float32(15.0))
+    lo_h = np.float16(lo)
+    sc_h = np.float16(scale)
+    lo32 = np.float32(lo_h)
+    sc32 = np.float32(sc_h)
+    if sc32 == 0:
+        q = np.zeros(x.shape, dtype=np.uint8)
+    else:
+        q = np.clip(np.rint(np.float32(x - lo32) / sc32), 0, 15).astype(np.uint8)
+    return q, lo_h, sc_h
+
+
+def dequantize4(q, lo_h, sc_h):
+    """lo + code * scale in fp32 (multiply, then add, each rounded)."""
+    prod = np.float32(np.asarray(q, dtype=np.float32) * np.float32(sc_h))
+    return np.float32(np.float32(lo_h) + prod)
+
+
+def residual_encode(X: np.ndarray, kind: str, group: int = RESIDUAL_GROUP):
+    """Recursive 4-bit coding of the adjacent-loop residuals of ``X [T][N][H][D]``.
+
+    kind "k": groups of ``group`` consecutive tokens per (step, head, channel);
+    kind "v": groups of ``group`` consecutive channels per (step, head, token).
+    The last token group may be shorter.  Returns ``(codes, lo, scale, recon)``:
+    codes ``[T][H][N][D]`` uint8 in 0..15; lo/scale fp16 ``[T][H][ceil(N/g)][D]``
+    for keys, ``[T][H][N][D/g]`` for values; recon ``[T][N][H][D]`` fp32, the
+    reconstruction each step reads (Khat_t).
+    """
+    T, N, H, D = X.shape
+    if D % group:
+        raise ValueError("head_dim must be a multiple of the group")
+    codes = np.zeros((T, H, N, D), dtype=np.uint8)
+    ng = -(-N // group)
+    if kind == "k":
+        lo = np.zeros((T, H, ng, D), dtype=np.float16)
+        sc = np.zeros((T, H, ng, D), dtype=np.float16)
+    elif kind == "v":
+        lo = np.zeros((T, H, N, D // group), dtype=np.float16)
+        sc = np.zeros((T, H, N, D // group), dtype=np.float16)
+    else:
+        raise ValueError("kind must be 'k' or 'v'")
+    acc = np.zeros((N, H, D), dtype=np.float32)
+    recon = np.zeros((T, N, H, D), dtype=np.float32)
+    for t in range(T):
+        r = np.float32(np.asarray(X[t], dtype=np.float32) - acc)   # [N][H][D]
+        deq = np.zeros_like(r)
+        for h in range(H):
+            if kind == "k":
+                for g in range(ng):
+                    n0, n1 = g * group, min(N, (g + 1) * group)
+                    for d in range(D):
+                        q, l, c = quantize4_group(r[n0:n1, h, d])
+                        codes[t, h, n0:n1, d] = q
+                        lo[t, h, g, d], sc[t, h, g, d] = l, c
+                        deq[n0:n1, h, d] = dequantize4(q, l, c)
+            else:
+                for n in range(N):
+                    for g in range(D // group):
+                        d0, d1 = g * group, (g + 1) * group
+                        q, l, c = quantize4_group(r[n, h, d0:d1])
+                        codes[t, h, n, d0:d1] = q
+                        lo[t, h, n, g], sc[t, h, n, g] = l, c
+                        deq[n, h, d0:d1] = dequantize4(q, l, c)
+        acc = np.float32(acc + deq)
+        recon[t] = acc
+    return codes, lo, sc, recon
+
+
+def residual_reconstruct(codes, lo, sc, kind: str, loop_step: int, group: int = RESIDUAL_GROUP):
+    """Khat_t ``[N][H][D]`` fp32 from stored codes: the dequantized residuals
+    of steps 0..t added in step order (fp32)."""
+    T, H, N, D = codes.shape
+    acc = np.zeros((N, H, D), dtype=np.float32)
+    for t in range(loop_step + 1):
+        for h in range(H):
+            if kind == "k":
+                lo_e = np.repeat(lo[t, h], group, axis=0)[:N]          # [N][D]
+                sc_e = np.repeat(sc[t, h], group, axis=0)[:N]
+            else:
+                lo_e = np.repeat(lo[t, h], group, axis=1)              # [N][D]
+                sc_e = np.repeat(sc[t, h], group, axis=1)
+            acc[:, h, :] = np.float32(acc[:, h, :] + dequantize4(codes[t, h], lo_e, sc_e))
+    return acc
+
+
+def residual_decode_attention(q, loop_step, k_codes, k_lo, k_sc, v_codes, v_lo, v_sc, scale):
+    """Decode attention of one request at loop step t over the reconstructed
+    residual-coded cache (every token quantized); q ``[Hq][D]``; returns
+    ``(o [Hq][D], lse [Hq])`` in fp64, query head hq reading KV head
+    hq // (Hq / H)."""
+    q = np.asarray(q, dtype=np.float64)
+    Hq = q.shape[0]
+    K = residual_reconstruct(k_codes, k_lo, k_sc, "k", loop_step)
+    V = residual_reconstruct(v_codes, v_lo, v_sc, "v", loop_step)
+    H = K.shape[1]
+    group = Hq // H
+    out = np.empty(q.shape, dtype=np.float64)
+    lse = np.empty(Hq, dtype=np.float64)
+    for hq in range(Hq):
+        out[hq], lse[hq] = attention(q[hq], K[:, hq // group, :], V[:, hq // group, :], scale)
+    return out, lse
+
+
+def residual_bits_per_element(group: int = RESIDUAL_GROUP) -> float:
+    """4 code bits plus an fp16 min and an fp16 scale shared by ``group``
+    elements."""
+    return 4.0 + 32.0 / group

@@ -499,3 +499,86 @@ def test_codebook_grad_zero_at_target_and_empty_body():
     np.testing.assert_allclose(out, ref, rtol=1e-13)
     assert loss == pytest.approx(2.0 * float(np.sum((ref - 1.0) ** 2)), rel=1e-13)
     assert not gk.any() and not gv.any()
+
+
+# ------------------------------------------- KV-residual 4-bit quantization
+
+def test_quantize4_grid_values_are_exact():
+    """Values on the 16-level grid of an fp16-representable min and scale
+    come back exactly, with their level as the code; the extremes are codes
+    0 and 15."""
+    lo, sc = np.float16(-1.25), np.float16(0.125)
+    levels = np.array([0, 15, 3, 7, 7, 12, 1, 15, 0, 9], dtype=np.uint8)
+    x = np.float32(lo) + levels.astype(np.float32) * np.float32(sc)
+    q, l, c = O.quantize4_group(x)
+    assert l == lo and c == sc
+    np.testing.assert_array_equal(q, levels)
+    np.testing.assert_array_equal(O.dequantize4(q, l, c), x)
+    # half-way values round to the even level
+    half = np.array([0, 15, 2.5, 3.5, 10.5], dtype=np.float32)
+    q, _, _ = O.quantize4_group(np.float32(lo) + half * np.float32(sc))
+    np.testing.assert_array_equal(q, [0, 15, 2, 4, 10])
+
+
+def test_quantize4_error_bound_and_constant_group():
+    """|x - dequant| is at most half a step plus the fp16 rounding of min and
+    scale (times the largest code); a constant group has scale 0, codes 0 and
+    reconstructs to its fp16-rounded value."""
+    rng = np.random.default_rng(700)
+    for _ in range(200):
+        x = (rng.standard_normal(32) * rng.uniform(0.01, 10)).astype(np.float32)
+        q, l, c = O.quantize4_group(x)
+        lo, hi = float(x.min()), float(x.max())
+        scale = np.float32(np.float32(hi - lo) / np.float32(15))
+        bound = 0.5 * float(c) + abs(float(l) - lo) + 15 * abs(float(c) - float(scale)) + 1e-6 * max(abs(lo), abs(hi))
+        assert np.max(np.abs(O.dequantize4(q, l, c) - x)) <= bound
+        assert q.max() <= 15
+    q, l, c = O.quantize4_group(np.full(32, 0.3, dtype=np.float32))
+    assert c == 0 and not q.any() and np.all(O.dequantize4(q, l, c) == np.float32(np.float16(0.3)))
+
+
+def test_residual_reconstruction_telescopes():
+    """Step 0 codes K_0 itself; the reconstruction read at step t is the sum of
+    the dequantized residuals of steps 0..t, and equals the encoder's running
+    reconstruction; keys group tokens (ragged last group), values channels."""
+    X = synth.loop_correlated(seed=710, n_loop=4, n_tokens=45, n_heads=2, head_dim=64)
+    for kind in ("k", "v"):
+        codes, lo, sc, recon = O.residual_encode(X, kind)
+        assert codes.max() <= 15
+        if kind == "k":
+            assert lo.shape == (4, 2, 2, 64)
+        else:
+            assert lo.shape == (4, 2, 45, 2)
+        for t in range(4):
+            np.testing.assert_array_equal(O.residual_reconstruct(codes, lo, sc, kind, t), recon[t])
+        # step 0 alone is plain 4-bit coding of K_0
+        c0, l0, s0, r0 = O.residual_encode(X[:1], kind)
+        np.testing.assert_array_equal(r0[0], recon[0])
+
+
+def test_residual_coding_beats_per_step_coding_on_loop_correlated_data():
+    """FlashLoop page, Figure 2 (c): recursively coding adjacent-loop residuals
+    reconstructs a loop-correlated cache with lower error than coding every
+    loop step's K/V on its own at the same bits."""
+    X = synth.loop_correlated(seed=720, n_loop=4, n_tokens=96, n_heads=2, head_dim=64, rho=0.95)
+    for kind in ("k", "v"):
+        _, _, _, recon = O.residual_encode(X, kind)
+        err_res = np.mean((recon[1:] - X[1:]) ** 2)
+        err_ind = 0.0
+        for t in range(1, 4):
+            _, _, _, r = O.residual_encode(X[t:t + 1], kind)
+            err_ind += np.mean((r[0] - X[t]) ** 2) / 3
+        assert err_res < err_ind, (kind, err_res, err_ind)
+
+
+def test_residual_decode_is_attention_over_the_reconstruction():
+    X = synth.loop_correlated(seed=730, n_loop=4, n_tokens=70, n_heads=1, head_dim=64)
+    Y = synth.loop_correlated(seed=731, n_loop=4, n_tokens=70, n_heads=1, head_dim=64)
+    kc, kl, ks, kr = O.residual_encode(X, "k")
+    vc, vl, vs, vr = O.residual_encode(Y, "v")
+    q = np.random.default_rng(732).standard_normal((2, 64))
+    for t in (0, 3):
+        o, lse = O.residual_decode_attention(q, t, kc, kl, ks, vc, vl, vs, 0.125)
+        for hq in range(2):
+            np.testing.assert_allclose(o[hq], _sdpa(q[hq], kr[t][:, 0], vr[t][:, 0], 0.125), rtol=1e-12, atol=1e-12)
+    assert O.residual_bits_per_element() == 5.0
