@@ -468,6 +468,80 @@ LOOPVQ_API loopvq_status loopvq_codebook_grad(const loopvq_codebook_desc* desc, 
                                               float* gradK, float* gradV, float* loss_out,
                                               uint32_t* fault_bits, loopvq_stream_t stream);
 
+/* ------------------------------ adjacent-loop KV-residual quantization */
+
+/*
+ * Second workload on the same loop axis (FlashLoop page, thelatestinai.com:
+ * "Figure 2 (c)", "Figure 3 (c-d)", "Table 2", "Figure 4"): the K/V residual
+ * between adjacent loop steps is coded with 4 bits.  Step 0 codes K_0; step t
+ * codes R_t = K_t - Khat_{t-1} (the previous step's reconstruction), and
+ * Khat_t = Khat_{t-1} + Q(R_t).  Q is KIVI's 4-bit asymmetric quantizer with
+ * an fp16 minimum and an fp16 scale per group of 32 values: keys are grouped
+ * per channel over 32 consecutive tokens, values per token over 32
+ * consecutive channels (5 bits per element with the parameters).  Every
+ * decision is taken in fp32 with separately rounded operations:
+ *   scale = (max - min) / 15;  min_h, scale_h = fp16(min), fp16(scale)
+ *   code  = scale_h == 0 ? 0 : clamp(rint((x - min_h) / scale_h), 0, 15)
+ *   dequant = min_h + code * scale_h
+ * Pools (pool_tokens a multiple of 32):
+ *   codes       [T][H][pool_tokens][D/2] uint8, channel 2i in the low nibble
+ *   key params  [T][H][pool_tokens/32][D] (min, scale) fp16 pairs
+ *   value params[T][H][pool_tokens][D/32] (min, scale) fp16 pairs
+ * A request's tokens start at a pool position that is a multiple of 32.
+ */
+typedef struct {
+  int32_t n_loop;      /* T */
+  int32_t n_heads_kv;  /* H */
+  int32_t n_heads_q;   /* Hq, a multiple of H */
+  int32_t head_dim;    /* D: 64 or 128 */
+} loopvq_residual_desc;
+
+/* Bytes of one codes pool / one parameter pool for pool_tokens tokens (0 if
+ * the descriptor is invalid or pool_tokens is not a positive multiple of 32). */
+LOOPVQ_API size_t loopvq_residual_codes_bytes(const loopvq_residual_desc* desc, int64_t pool_tokens);
+LOOPVQ_API size_t loopvq_residual_params_bytes(const loopvq_residual_desc* desc, loopvq_kind kind,
+                                               int64_t pool_tokens);
+
+/*
+ * Codes all T loop steps of n_tokens tokens of x (keys or values, element
+ * (t, n, h, d) at t*stride_t + n*stride_n + h*stride_h + d, bf16 or fp32)
+ * into the pools at positions tok_off .. tok_off + n_tokens - 1 (tok_off a
+ * multiple of 32; a last key group shorter than 32 tokens takes its min and
+ * scale over the tokens present).  One kernel on `stream`.
+ */
+LOOPVQ_API loopvq_status loopvq_residual_encode(const loopvq_residual_desc* desc, loopvq_kind kind, const void* x,
+                                                loopvq_dtype x_dtype, int64_t n_tokens, int64_t stride_t,
+                                                int64_t stride_n, int64_t stride_h, uint8_t* codes, void* params,
+                                                int64_t tok_off, int64_t pool_tokens, loopvq_stream_t stream);
+
+/* Workspace bytes of loopvq_residual_decode_attn (0 if invalid). */
+LOOPVQ_API size_t loopvq_residual_decode_workspace_bytes(const loopvq_residual_desc* desc, int32_t batch,
+                                                         int32_t max_ctx_len);
+
+/*
+ * Decode attention at loop step t over the residual-coded cache: request r's
+ * ctx_len[r] tokens at pool positions tok_off[r] .. (every token coded, no
+ * bf16 window); each token's key and value rows are rebuilt from the t+1
+ * residual planes added in step order (the encoder's reconstruction, bit
+ * for bit) and o = softmax(softmax_scale * q . k) v in fp32.
+ *   ctx_len, tok_off : device [batch] int32 / int64.
+ *   q [batch][Hq][D] in q_dtype; out [batch][Hq][D] fp32; lse_out nullable.
+ *   codesK/V  : 8-byte aligned; paramsK 16-byte, paramsV 4-byte aligned.
+ *   workspace : zero-filled before its first use (status word, split
+ *               counters, partials), 256-byte aligned.
+ * A request with ctx_len 0 gets a zero output and lse -inf; a context or
+ * offset out of range sets a LOOPVQ_FAULT_* bit in the workspace status word
+ * (loopvq_read_device_status) and gives that request a zero output.
+ */
+LOOPVQ_API loopvq_status loopvq_residual_decode_attn(const loopvq_residual_desc* desc, int32_t batch,
+                                                     int32_t max_ctx_len, const int32_t* ctx_len,
+                                                     const int64_t* tok_off, int64_t pool_tokens,
+                                                     const uint8_t* codesK, const void* paramsK,
+                                                     const uint8_t* codesV, const void* paramsV, const void* q,
+                                                     loopvq_dtype q_dtype, int32_t loop_step, float softmax_scale,
+                                                     float* out, float* lse_out, void* workspace,
+                                                     size_t workspace_bytes, loopvq_stream_t stream);
+
 /* -------------------------------------------------- dense bf16 comparator */
 
 /* Workspace bytes of loopvq_dense_decode_attn. */

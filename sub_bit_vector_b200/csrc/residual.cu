@@ -1,0 +1,450 @@
+// Adjacent-loop KV-residual 4-bit quantization and decode attention (sm_100a).
+//
+// FlashLoop page (thelatestinai.com; "Figure 2 (c)", "Figure 3 (c-d)",
+// "Table 2", "Figure 4"): K/V residuals between adjacent loop steps shrink
+// with depth, and recursively quantizing them reconstructs the cache better
+// than quantizing every loop's complete K/V; the method uses 4-bit residuals
+// along the axes of per-loop KIVI4.  Step 0 codes K_0; step t codes
+// R_t = K_t - Khat_{t-1}, the residual against the previous reconstruction,
+// and Khat_t = Khat_{t-1} + Q(R_t).  Q is KIVI's quantizer: 16 levels, an
+// fp16 minimum and an fp16 scale per group of 32 values; keys are grouped
+// per channel over 32 consecutive tokens, values per token over 32
+// consecutive channels.  Every decision is taken in fp32 with separately
+// rounded operations (no contraction), so the codes are reproducible bit for
+// bit:  scale = (max - min) / 15, code = clamp(rint((x - min_h) / scale_h),
+// 0, 15), dequant = min_h + code * scale_h.
+//
+// Pool layouts (pool_tokens a multiple of 32, a request's tokens start at a
+// multiple of 32 so key groups are pool-aligned):
+//   codes         [T][H][pool_tokens][D/2]  two codes per byte, even channel low
+//   key params    [T][H][pool_tokens/32][D] half2 (min, scale)
+//   value params  [T][H][pool_tokens][D/32] half2 (min, scale)
+//
+// Decode at loop step t reconstructs each token's key and value rows from
+// the t+1 residual planes (added in step order, as the encoder did; eight
+// lanes per token, each with D/8 channels) and runs split-K attention with an
+// fp32 online softmax; the last split of a (request, head) merges the splits.
+
+#include <cuda_fp16.h>
+#include <math.h>
+
+#include "common.cuh"
+
+namespace loopvq {
+
+constexpr int kRG = 32;  // values per quantization group
+
+struct ResGeo {
+  int T, H, Hq, D;
+};
+
+static loopvq_status res_geo(const loopvq_residual_desc* d, ResGeo* g) {
+  if (!d || d->n_loop < 1 || d->n_heads_kv < 1 || d->n_heads_q < 1 || d->n_heads_q % d->n_heads_kv)
+    return LOOPVQ_ERR_INVALID_ARG;
+  if (d->head_dim != 64 && d->head_dim != 128) return LOOPVQ_ERR_UNSUPPORTED;
+  g->T = d->n_loop;
+  g->H = d->n_heads_kv;
+  g->Hq = d->n_heads_q;
+  g->D = d->head_dim;
+  return LOOPVQ_OK;
+}
+
+// One 4-bit decision of KIVI's quantizer on x given the group's stored min
+// and scale (already rounded to fp16 and back).
+__device__ __forceinline__ uint32_t q4(float x, float lo, float sc) {
+  if (sc == 0.f) return 0u;
+  const float v = rintf(__fdiv_rn(__fsub_rn(x, lo), sc));
+  return (uint32_t)fminf(fmaxf(v, 0.f), 15.f);
+}
+__device__ __forceinline__ float dq4(uint32_t q, float lo, float sc) { return __fadd_rn(lo, __fmul_rn((float)q, sc)); }
+
+struct ResEncParams {
+  const void* x;
+  int x_bf16;
+  int64_t st, sn, sh;
+  int64_t n_tokens, tok_off, pool;
+  int T, H, D;
+  uint8_t* codes;
+  __half2* params;
+};
+
+__device__ __forceinline__ float ld_x(const ResEncParams& p, int t, int64_t n, int h, int d) {
+  const int64_t e = (int64_t)t * p.st + n * p.sn + (int64_t)h * p.sh + d;
+  return p.x_bf16 ? __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(p.x)[e])
+                  : reinterpret_cast<const float*>(p.x)[e];
+}
+
+// Keys: one warp per (token group, head, 32-channel block); lane = channel.
+// The running reconstruction of the group's 32 tokens lives in shared memory
+// (lane = bank); each step reads the group twice (min/max, then codes; the
+// second read hits L1).
+constexpr int kREncWarps = 8;
+__global__ void __launch_bounds__(kREncWarps * 32) res_encode_keys(const ResEncParams p) {
+  __shared__ float accs[kREncWarps][kRG][32];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int64_t wid = (int64_t)blockIdx.x * kREncWarps + warp;
+  const int cblocks = p.D / 32;
+  const int64_t n_groups = (p.n_tokens + kRG - 1) / kRG;
+  if (wid >= n_groups * p.H * cblocks) return;
+  const int cb = (int)(wid % cblocks);
+  const int h = (int)((wid / cblocks) % p.H);
+  const int64_t g = wid / ((int64_t)cblocks * p.H);
+  const int d = cb * 32 + lane;
+  const int64_t n0 = g * kRG;
+  const int gl = (int)min((int64_t)kRG, p.n_tokens - n0);
+  float (*acc)[32] = accs[warp];
+  for (int i = 0; i < kRG; ++i) acc[i][lane] = 0.f;
+  const int64_t pg = (p.tok_off + n0) / kRG;  // pool group
+  for (int t = 0; t < p.T; ++t) {
+    float lo = INFINITY, hi = -INFINITY;
+#pragma unroll 4
+    for (int i = 0; i < gl; ++i) {
+      const float r = __fsub_rn(ld_x(p, t, n0 + i, h, d), acc[i][lane]);
+      lo = fminf(lo, r);
+      hi = fmaxf(hi, r);
+    }
+    const __half lo_h = __float2half_rn(lo);
+    const __half sc_h = __float2half_rn(__fdiv_rn(__fsub_rn(hi, lo), 15.f));
+    const float lo32 = __half2float(lo_h), sc32 = __half2float(sc_h);
+    p.params[(((int64_t)t * p.H + h) * (p.pool / kRG) + pg) * p.D + d] = __halves2half2(lo_h, sc_h);
+    uint8_t* crow = p.codes + (((int64_t)t * p.H + h) * p.pool + p.tok_off + n0) * (p.D / 2) + d / 2;
+#pragma unroll 4
+    for (int i = 0; i < gl; ++i) {   // gl is warp-uniform: every lane takes the shuffle
+      const float r = __fsub_rn(ld_x(p, t, n0 + i, h, d), acc[i][lane]);
+      const uint32_t q = q4(r, lo32, sc32);
+      const uint32_t q_odd = __shfl_down_sync(0xffffffffu, q, 1);
+      acc[i][lane] = __fadd_rn(acc[i][lane], dq4(q, lo32, sc32));
+      if (!(lane & 1)) crow[(int64_t)i * (p.D / 2)] = (uint8_t)(q | (q_odd << 4));
+    }
+  }
+}
+
+// Values: one warp per (token, head, 32-channel group); lane = channel, the
+// group's min and max by shuffles.
+__global__ void __launch_bounds__(256) res_encode_values(const ResEncParams p) {
+  const int lane = threadIdx.x & 31;
+  const int64_t wid = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int cgroups = p.D / kRG;
+  if (wid >= p.n_tokens * p.H * cgroups) return;
+  const int cg = (int)(wid % cgroups);
+  const int h = (int)((wid / cgroups) % p.H);
+  const int64_t n = wid / ((int64_t)cgroups * p.H);
+  const int d = cg * kRG + lane;
+  const int64_t pos = p.tok_off + n;
+  float acc = 0.f;
+  for (int t = 0; t < p.T; ++t) {
+    const float r = __fsub_rn(ld_x(p, t, n, h, d), acc);
+    float lo = r, hi = r;
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) {
+      lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+      hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+    }
+    const __half lo_h = __float2half_rn(lo);
+    const __half sc_h = __float2half_rn(__fdiv_rn(__fsub_rn(hi, lo), 15.f));
+    const float lo32 = __half2float(lo_h), sc32 = __half2float(sc_h);
+    if (lane == 0) p.params[(((int64_t)t * p.H + h) * p.pool + pos) * cgroups + cg] = __halves2half2(lo_h, sc_h);
+    const uint32_t q = q4(r, lo32, sc32);
+    const uint32_t q_odd = __shfl_down_sync(0xffffffffu, q, 1);
+    acc = __fadd_rn(acc, dq4(q, lo32, sc32));
+    if (!(lane & 1)) p.codes[(((int64_t)t * p.H + h) * p.pool + pos) * (p.D / 2) + d / 2] = (uint8_t)(q | (q_odd << 4));
+  }
+}
+
+// ------------------------------------------------------------------ decode
+constexpr int kRW = 16;                 // warps per CTA
+constexpr int kRThreads = kRW * 32;
+
+struct ResDecParams {
+  int T, H, Hq, D, loop_step, max_ctx, split_len, max_splits;
+  const int32_t* ctx_len;
+  const int64_t* tok_off;
+  int64_t pool;
+  const uint8_t* ck;
+  const __half2* pk;
+  const uint8_t* cv;
+  const __half2* pv;
+  const void* q;
+  int q_bf16;
+  float scale_log2;
+  float* out;
+  float* lse;
+  uint32_t* status;
+  uint32_t* tickets;
+  float* partials;
+};
+
+// Eight lanes share a token (lane group g = lane / 8 of a warp takes token
+// base + g): lane i of the group owns channels i*CPL .. i*CPL+CPL-1, so one
+// lane reads CPL/2 bytes of codes per plane, its CPL key (min, scale) pairs
+// (shared by the 32 tokens of a key group: L1 hits) and one value pair.
+constexpr int kRLanesPerTok = 8;
+constexpr int kRTokPerWarp = 32 / kRLanesPerTok;
+
+template <int CPL>
+__device__ __forceinline__ void res_row(const ResDecParams& p, int h, int64_t pos, int li, float (&k)[CPL],
+                                        float (&v)[CPL]) {
+  constexpr int D = CPL * kRLanesPerTok;
+#pragma unroll
+  for (int i = 0; i < CPL; ++i) k[i] = v[i] = 0.f;
+#pragma unroll 4
+  for (int s = 0; s <= p.loop_step; ++s) {   // unrolled so that the planes' loads issue together
+    const int64_t plane = (int64_t)s * p.H + h;
+    const int64_t row = (plane * p.pool + pos) * (D / 2) + li * (CPL / 2);
+    uint32_t kc[CPL / 8], vc[CPL / 8];
+    if constexpr (CPL == 16) {
+      const uint2 a = __ldg(reinterpret_cast<const uint2*>(p.ck + row));
+      const uint2 b = __ldg(reinterpret_cast<const uint2*>(p.cv + row));
+      kc[0] = a.x; kc[1] = a.y; vc[0] = b.x; vc[1] = b.y;
+    } else {
+      kc[0] = __ldg(reinterpret_cast<const uint32_t*>(p.ck + row));
+      vc[0] = __ldg(reinterpret_cast<const uint32_t*>(p.cv + row));
+    }
+    const uint4* kp = reinterpret_cast<const uint4*>(p.pk + (plane * (p.pool / kRG) + pos / kRG) * D + li * CPL);
+    const float2 vpar = __half22float2(__ldg(p.pv + (plane * p.pool + pos) * (D / kRG) + (li * CPL) / kRG));
+#pragma unroll
+    for (int w = 0; w < CPL / 4; ++w) {
+      const uint4 pw = __ldg(kp + w);   // 4 (min, scale) pairs
+      const uint32_t pr[4] = {pw.x, pw.y, pw.z, pw.w};
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int i = w * 4 + u;
+        const float2 kpar = __half22float2(*reinterpret_cast<const __half2*>(&pr[u]));
+        const uint32_t ck = (kc[i >> 3] >> (4 * (i & 7))) & 15u;
+        const uint32_t cv = (vc[i >> 3] >> (4 * (i & 7))) & 15u;
+        k[i] = __fadd_rn(k[i], dq4(ck, kpar.x, kpar.y));
+        v[i] = __fadd_rn(v[i], dq4(cv, vpar.x, vpar.y));
+      }
+    }
+  }
+}
+
+template <int CPL>
+__global__ void __launch_bounds__(kRThreads) res_decode_kernel(const ResDecParams p) {
+  constexpr int D = CPL * kRLanesPerTok;
+  __shared__ float wpart[kRW][D + 2];
+  __shared__ float csm[2 * kMaxCombineSplits + kRThreads];
+  __shared__ int flag;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int grp = lane / kRLanesPerTok, li = lane % kRLanesPerTok;
+  const int split = blockIdx.x, hq = blockIdx.y, r = blockIdx.z;
+  const int h = hq / (p.Hq / p.H);
+  const size_t unit = (size_t)r * p.Hq + hq;
+  int ctx = __ldg(p.ctx_len + r);
+  const int64_t off = __ldg(p.tok_off + r);
+  if (ctx < 0 || ctx > p.max_ctx) {
+    if (tid == 0 && split == 0) set_fault(p.status, LOOPVQ_FAULT_CTX_RANGE);
+    ctx = 0;
+  }
+  if (ctx > 0 && (off < 0 || (off % kRG) || off + ctx > p.pool)) {
+    if (tid == 0 && split == 0) set_fault(p.status, LOOPVQ_FAULT_POOL_RANGE);
+    ctx = 0;
+  }
+  const int n_splits = (ctx + p.split_len - 1) / p.split_len;
+  if (ctx == 0) {
+    if (split == 0) {
+      for (int d = tid; d < D; d += blockDim.x) p.out[unit * D + d] = 0.f;
+      if (p.lse && tid == 0) p.lse[unit] = -INFINITY;
+    }
+    return;
+  }
+  if (split >= n_splits) return;
+  const int t0 = split * p.split_len;
+  const int t1 = min(ctx, t0 + p.split_len);
+
+  float qv[CPL];
+#pragma unroll
+  for (int i = 0; i < CPL; ++i) {
+    const size_t qi = unit * D + li * CPL + i;
+    qv[i] = (p.q_bf16 ? __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(p.q)[qi])
+                      : reinterpret_cast<const float*>(p.q)[qi]) *
+            p.scale_log2;
+  }
+  float m = -INFINITY, l = 0.f, o[CPL];
+#pragma unroll
+  for (int i = 0; i < CPL; ++i) o[i] = 0.f;
+  for (int base = t0 + warp * kRTokPerWarp; base < t1; base += kRW * kRTokPerWarp) {
+    const int tok = base + grp;
+    float kf[CPL], vf[CPL];
+    res_row<CPL>(p, h, off + min(tok, t1 - 1), li, kf, vf);  // past the end: a valid row, masked below
+    float a = 0.f;
+#pragma unroll
+    for (int i = 0; i < CPL; ++i) a = fmaf(qv[i], kf[i], a);
+#pragma unroll
+    for (int x = kRLanesPerTok / 2; x >= 1; x >>= 1) a += __shfl_xor_sync(0xffffffffu, a, x);
+    const float sc = tok < t1 ? a : -INFINITY;
+    const float mn = fmaxf(m, sc);
+    if (mn != -INFINITY) {
+      const float corr = exp2f(m - mn);
+      const float pw = exp2f(sc - mn);
+      l = fmaf(l, corr, pw);
+#pragma unroll
+      for (int i = 0; i < CPL; ++i) o[i] = fmaf(o[i], corr, pw * vf[i]);
+      m = mn;
+    }
+  }
+  // merge the warp's four token groups (lanes li, li + 8, li + 16, li + 24)
+#pragma unroll
+  for (int x = kRLanesPerTok; x < 32; x <<= 1) {
+    const float mo = __shfl_xor_sync(0xffffffffu, m, x);
+    const float lo_ = __shfl_xor_sync(0xffffffffu, l, x);
+    const float mn = fmaxf(m, mo);
+    const float ca = m == -INFINITY ? 0.f : exp2f(m - mn);
+    const float cb = mo == -INFINITY ? 0.f : exp2f(mo - mn);
+#pragma unroll
+    for (int i = 0; i < CPL; ++i) {
+      const float oo = __shfl_xor_sync(0xffffffffu, o[i], x);
+      o[i] = o[i] * ca + oo * cb;
+    }
+    l = l * ca + lo_ * cb;
+    m = mn;
+  }
+  if (grp == 0) {
+#pragma unroll
+    for (int i = 0; i < CPL; ++i) wpart[warp][li * CPL + i] = o[i];
+    if (li == 0) { wpart[warp][D] = m; wpart[warp][D + 1] = l; }
+  }
+  __syncthreads();
+  float* part = p.partials + (unit * p.max_splits + split) * (size_t)(D + 4);
+  float M = -INFINITY;
+  for (int w = 0; w < kRW; ++w) M = fmaxf(M, wpart[w][D]);
+  for (int d = tid; d < D + 2; d += blockDim.x) {
+    float acc = 0.f;
+    if (d != D) {
+      for (int w = 0; w < kRW; ++w) {
+        const float mw = wpart[w][D];
+        if (mw != -INFINITY) acc += wpart[w][d] * exp2f(mw - M);
+      }
+    }
+    part[d] = (d == D) ? M : acc;
+  }
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) flag = (atomicAdd(p.tickets + unit, 1u) == (uint32_t)(n_splits - 1)) ? 1 : 0;
+  __syncthreads();
+  if (flag) {
+    __threadfence();
+    combine_splits(p.partials + unit * p.max_splits * (size_t)(D + 4), n_splits, D, p.out + unit * D, 0,
+                   p.lse ? p.lse + unit : nullptr, csm, tid, kRThreads, BlockSync{});
+    if (tid == 0) atomicExch(p.tickets + unit, 0u);
+  }
+}
+
+static void res_plan(int64_t units, int max_ctx, int n_sm, int* split_len, int* max_splits) {
+  int s = (int)(n_sm / (units > 0 ? units : 1));
+  const int cap = (max_ctx + 255) / 256;
+  if (s > cap) s = cap;
+  if (s < 1) s = 1;
+  int len = (max_ctx + s - 1) / s;
+  if (len < 1) len = 1;
+  *split_len = len;
+  *max_splits = max_ctx > 0 ? (max_ctx + len - 1) / len : 1;
+}
+
+}  // namespace loopvq
+
+using namespace loopvq;
+
+extern "C" size_t loopvq_residual_codes_bytes(const loopvq_residual_desc* desc, int64_t pool_tokens) {
+  ResGeo g;
+  if (res_geo(desc, &g) != LOOPVQ_OK || pool_tokens <= 0 || (pool_tokens % kRG)) return 0;
+  return (size_t)g.T * g.H * pool_tokens * (g.D / 2);
+}
+
+extern "C" size_t loopvq_residual_params_bytes(const loopvq_residual_desc* desc, loopvq_kind kind,
+                                               int64_t pool_tokens) {
+  ResGeo g;
+  if (res_geo(desc, &g) != LOOPVQ_OK || pool_tokens <= 0 || (pool_tokens % kRG)) return 0;
+  if (kind == LOOPVQ_KEYS) return (size_t)g.T * g.H * (pool_tokens / kRG) * g.D * sizeof(__half2);
+  if (kind == LOOPVQ_VALUES) return (size_t)g.T * g.H * pool_tokens * (g.D / kRG) * sizeof(__half2);
+  return 0;
+}
+
+extern "C" loopvq_status loopvq_residual_encode(const loopvq_residual_desc* desc, loopvq_kind kind, const void* x,
+                                                loopvq_dtype x_dtype, int64_t n_tokens, int64_t stride_t,
+                                                int64_t stride_n, int64_t stride_h, uint8_t* codes, void* params,
+                                                int64_t tok_off, int64_t pool_tokens, loopvq_stream_t stream) {
+  ResGeo g;
+  loopvq_status st = res_geo(desc, &g);
+  if (st != LOOPVQ_OK) return st;
+  if (kind != LOOPVQ_KEYS && kind != LOOPVQ_VALUES) return LOOPVQ_ERR_INVALID_ARG;
+  if (x_dtype != LOOPVQ_F32 && x_dtype != LOOPVQ_BF16) return LOOPVQ_ERR_INVALID_ARG;
+  if (n_tokens < 0 || tok_off < 0 || (tok_off % kRG) || pool_tokens <= 0 || (pool_tokens % kRG) ||
+      tok_off + n_tokens > pool_tokens)
+    return LOOPVQ_ERR_INVALID_ARG;
+  if (stride_t < 0 || stride_n < 0 || stride_h < 0) return LOOPVQ_ERR_INVALID_ARG;
+  if (!x || !codes || !params || ((uintptr_t)params & 3)) return LOOPVQ_ERR_INVALID_ARG;
+  if (n_tokens == 0) return LOOPVQ_OK;
+  ResEncParams p;
+  p.x = x; p.x_bf16 = x_dtype == LOOPVQ_BF16;
+  p.st = stride_t; p.sn = stride_n; p.sh = stride_h;
+  p.n_tokens = n_tokens; p.tok_off = tok_off; p.pool = pool_tokens;
+  p.T = g.T; p.H = g.H; p.D = g.D;
+  p.codes = codes; p.params = (__half2*)params;
+  const int64_t warps = kind == LOOPVQ_KEYS ? ((n_tokens + kRG - 1) / kRG) * g.H * (g.D / 32)
+                                            : n_tokens * g.H * (g.D / kRG);
+  const int64_t blocks = (warps + 7) / 8;
+  if (blocks > 0x7fffffffLL) return LOOPVQ_ERR_UNSUPPORTED;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (kind == LOOPVQ_KEYS)
+    res_encode_keys<<<(unsigned)blocks, kREncWarps * 32, 0, s>>>(p);
+  else
+    res_encode_values<<<(unsigned)blocks, 256, 0, s>>>(p);
+  return cudaGetLastError() == cudaSuccess ? LOOPVQ_OK : LOOPVQ_ERR_CUDA;
+}
+
+extern "C" size_t loopvq_residual_decode_workspace_bytes(const loopvq_residual_desc* desc, int32_t batch,
+                                                         int32_t max_ctx_len) {
+  ResGeo g;
+  if (res_geo(desc, &g) != LOOPVQ_OK || batch < 1 || max_ctx_len < 0) return 0;
+  int len, ms;
+  res_plan((int64_t)batch * g.Hq, max_ctx_len, 1024, &len, &ms);
+  return ws_layout((int64_t)batch * g.Hq, ms, g.D).total;
+}
+
+extern "C" loopvq_status loopvq_residual_decode_attn(const loopvq_residual_desc* desc, int32_t batch,
+                                                     int32_t max_ctx_len, const int32_t* ctx_len,
+                                                     const int64_t* tok_off, int64_t pool_tokens,
+                                                     const uint8_t* codesK, const void* paramsK,
+                                                     const uint8_t* codesV, const void* paramsV, const void* q,
+                                                     loopvq_dtype q_dtype, int32_t loop_step, float softmax_scale,
+                                                     float* out, float* lse_out, void* workspace,
+                                                     size_t workspace_bytes, loopvq_stream_t stream) {
+  ResGeo g;
+  loopvq_status st = res_geo(desc, &g);
+  if (st != LOOPVQ_OK) return st;
+  if (batch < 1 || max_ctx_len < 0 || pool_tokens <= 0 || (pool_tokens % kRG)) return LOOPVQ_ERR_INVALID_ARG;
+  if (loop_step < 0 || loop_step >= g.T) return LOOPVQ_ERR_INVALID_ARG;
+  if (q_dtype != LOOPVQ_F32 && q_dtype != LOOPVQ_BF16) return LOOPVQ_ERR_INVALID_ARG;
+  if (!(softmax_scale == softmax_scale)) return LOOPVQ_ERR_INVALID_ARG;
+  if (!ctx_len || !tok_off || !codesK || !paramsK || !codesV || !paramsV || !q || !out || !workspace)
+    return LOOPVQ_ERR_INVALID_ARG;
+  if (((uintptr_t)paramsK & 15) || ((uintptr_t)paramsV & 3) || ((uintptr_t)codesK & 7) || ((uintptr_t)codesV & 7) ||
+      ((uintptr_t)workspace & 255))
+    return LOOPVQ_ERR_INVALID_ARG;
+  if (workspace_bytes < loopvq_residual_decode_workspace_bytes(desc, batch, max_ctx_len))
+    return LOOPVQ_ERR_WORKSPACE_TOO_SMALL;
+  if (batch > 65535 || g.Hq > 65535) return LOOPVQ_ERR_UNSUPPORTED;
+  const int64_t units = (int64_t)batch * g.Hq;
+  int len, ms;
+  res_plan(units, max_ctx_len, device_sm_count(), &len, &ms);
+  if (ms > kMaxCombineSplits) return LOOPVQ_ERR_UNSUPPORTED;
+  const WsLayout ws = ws_layout(units, ms, g.D);
+  ResDecParams p;
+  p.T = g.T; p.H = g.H; p.Hq = g.Hq; p.D = g.D; p.loop_step = loop_step; p.max_ctx = max_ctx_len;
+  p.split_len = len; p.max_splits = ms;
+  p.ctx_len = ctx_len; p.tok_off = tok_off; p.pool = pool_tokens;
+  p.ck = codesK; p.pk = (const __half2*)paramsK; p.cv = codesV; p.pv = (const __half2*)paramsV;
+  p.q = q; p.q_bf16 = q_dtype == LOOPVQ_BF16;
+  p.scale_log2 = softmax_scale * 1.4426950408889634f;
+  p.out = out; p.lse = lse_out;
+  p.status = (uint32_t*)workspace;
+  p.tickets = (uint32_t*)((uint8_t*)workspace + ws.tickets_off);
+  p.partials = (float*)((uint8_t*)workspace + ws.partials_off);
+  dim3 grid(ms, g.Hq, batch);
+  if (g.D == 128)
+    res_decode_kernel<16><<<grid, kRThreads, 0, (cudaStream_t)stream>>>(p);
+  else
+    res_decode_kernel<8><<<grid, kRThreads, 0, (cudaStream_t)stream>>>(p);
+  return cudaGetLastError() == cudaSuccess ? LOOPVQ_OK : LOOPVQ_ERR_CUDA;
+}

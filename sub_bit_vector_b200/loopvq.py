@@ -45,6 +45,8 @@ EXPORTED = [
     "loopvq_codebook_update_workspace_bytes", "loopvq_codebook_update", "loopvq_codebook_grad",
     "loopvq_decode_workspace_bytes", "loopvq_decode_attn", "loopvq_decode_attn_noalloc",
     "loopvq_decode_steps_workspace_bytes", "loopvq_decode_attn_steps",
+    "loopvq_residual_codes_bytes", "loopvq_residual_params_bytes", "loopvq_residual_encode",
+    "loopvq_residual_decode_workspace_bytes", "loopvq_residual_decode_attn",
     "loopvq_read_device_status",
     "loopvq_clear_device_status", "loopvq_dense_decode_workspace_bytes", "loopvq_dense_decode_attn",
 ]
@@ -60,6 +62,11 @@ class loopvq_codebook_desc(ctypes.Structure):
     _fields_ = [("n_loop", ctypes.c_int32), ("tc", ctypes.c_int32), ("n_heads_kv", ctypes.c_int32),
                 ("n_heads_q", ctypes.c_int32), ("head_dim", ctypes.c_int32), ("group_elems", ctypes.c_int32),
                 ("n_codes", ctypes.c_int32), ("cb_dtype", ctypes.c_int)]
+
+
+class loopvq_residual_desc(ctypes.Structure):
+    _fields_ = [("n_loop", ctypes.c_int32), ("n_heads_kv", ctypes.c_int32), ("n_heads_q", ctypes.c_int32),
+                ("head_dim", ctypes.c_int32)]
 
 
 class loopvq_cache_layout(ctypes.Structure):
@@ -80,6 +87,7 @@ def _load() -> ctypes.CDLL:
                                ctypes.c_float, ctypes.c_void_p)
     D = ctypes.POINTER(loopvq_codebook_desc)
     L = ctypes.POINTER(loopvq_cache_layout)
+    RD = ctypes.POINTER(loopvq_residual_desc)
     sig = {
         "loopvq_version": (ctypes.c_char_p, []),
         "loopvq_status_string": (ctypes.c_char_p, [ctypes.c_int]),
@@ -99,6 +107,13 @@ def _load() -> ctypes.CDLL:
                                                   P, P, P, P, SZ, P]),
         "loopvq_codebook_grad": (ctypes.c_int, [D, P, P, L, U8P, U8P, P, ctypes.c_int, I32, F, P, P, P, F, P, P,
                                                 P, P, P]),
+        "loopvq_residual_codes_bytes": (SZ, [RD, I64]),
+        "loopvq_residual_params_bytes": (SZ, [RD, ctypes.c_int, I64]),
+        "loopvq_residual_encode": (ctypes.c_int, [RD, ctypes.c_int, P, ctypes.c_int, I64, I64, I64, I64, U8P, P, I64,
+                                                  I64, P]),
+        "loopvq_residual_decode_workspace_bytes": (SZ, [RD, I32, I32]),
+        "loopvq_residual_decode_attn": (ctypes.c_int, [RD, I32, I32, P, P, I64, U8P, P, U8P, P, P, ctypes.c_int, I32,
+                                                       F, P, P, P, SZ, P]),
         "loopvq_decode_workspace_bytes": (SZ, [D, L]),
         "loopvq_decode_attn": (ctypes.c_int, [D, P, P, L, U8P, U8P, P, P, P, ctypes.c_int, I32, F, P,
                                               ctypes.c_int, P, P, SZ, P]),
@@ -271,6 +286,38 @@ def loopvq_codebook_grad(desc, cbK, cbV, layout, idxK_pool, idxV_pool, q, loop_s
         ctypes.byref(desc), _ptr(cbK), _ptr(cbV), ctypes.byref(layout), _ptr(idxK_pool), _ptr(idxV_pool), _ptr(q),
         _dtype_code(q), loop_step, softmax_scale, _ptr(out), _ptr(lse), _ptr(target), weight, _ptr(gradK),
         _ptr(gradV), _ptr(loss_out), _ptr(fault_bits), _stream(stream)))
+
+
+def make_residual_desc(n_loop, n_heads_kv, head_dim, n_heads_q=None) -> loopvq_residual_desc:
+    return loopvq_residual_desc(n_loop, n_heads_kv, n_heads_q or n_heads_kv, head_dim)
+
+
+def loopvq_residual_codes_bytes(desc, pool_tokens) -> int:
+    return _lib.loopvq_residual_codes_bytes(ctypes.byref(desc), pool_tokens)
+
+
+def loopvq_residual_params_bytes(desc, kind, pool_tokens) -> int:
+    return _lib.loopvq_residual_params_bytes(ctypes.byref(desc), kind, pool_tokens)
+
+
+def loopvq_residual_encode(desc, kind, x, n_tokens, stride_t, stride_n, stride_h, codes, params, tok_off,
+                           pool_tokens, stream=None, x_dtype=None) -> None:
+    xd = _dtype_code(x) if x_dtype is None else x_dtype
+    _check("loopvq_residual_encode", _lib.loopvq_residual_encode(
+        ctypes.byref(desc), kind, _ptr(x), xd, n_tokens, stride_t, stride_n, stride_h, _ptr(codes), _ptr(params),
+        tok_off, pool_tokens, _stream(stream)))
+
+
+def loopvq_residual_decode_workspace_bytes(desc, batch, max_ctx_len) -> int:
+    return _lib.loopvq_residual_decode_workspace_bytes(ctypes.byref(desc), batch, max_ctx_len)
+
+
+def loopvq_residual_decode_attn(desc, batch, max_ctx_len, ctx_len, tok_off, pool_tokens, codesK, paramsK, codesV,
+                                paramsV, q, loop_step, softmax_scale, out, lse_out, workspace, stream=None) -> None:
+    _check("loopvq_residual_decode_attn", _lib.loopvq_residual_decode_attn(
+        ctypes.byref(desc), batch, max_ctx_len, _ptr(ctx_len), _ptr(tok_off), pool_tokens, _ptr(codesK),
+        _ptr(paramsK), _ptr(codesV), _ptr(paramsV), _ptr(q), _dtype_code(q), loop_step, softmax_scale, _ptr(out),
+        _ptr(lse_out), _ptr(workspace), _nbytes(workspace), _stream(stream)))
 
 
 def loopvq_decode_workspace_bytes(desc, layout) -> int:

@@ -16,6 +16,9 @@ holds well under 2 GB on the device:
 - ``encode``  : loop-axis encode of a [4][32768][16][128] bf16 tensor at
                 Tc = 4, G = 16 (tensor-core kernel), 2 launches.
 - ``encode-f32``: the same tensor in fp32 (CUDA-core kernel), 2 launches.
+- ``residual``: adjacent-loop residual 4-bit coding of [4][32768][16][128]
+                bf16 keys and values, then one decode per loop step (4
+                launches of the decode kernel).
 - ``page``    : encode of one 8-token page out of a [4][16][320][128] bf16
                 window pool (few-token kernel), 4 launches.
 """
@@ -93,6 +96,29 @@ def _encode(dtype):
     print("encode faults", L.loopvq_read_encode_faults())
 
 
+def _residual():
+    T, N, H, D = 4, 32768, 16, 128
+    desc = L.make_residual_desc(T, H, D)
+    bufs = []
+    for kind in (L.LOOPVQ_KEYS, L.LOOPVQ_VALUES):
+        codes = torch.zeros(L.loopvq_residual_codes_bytes(desc, N), dtype=torch.uint8, device="cuda")
+        params = torch.zeros(L.loopvq_residual_params_bytes(desc, kind, N) // 2, dtype=torch.float16, device="cuda")
+        x = synth.device_normal(20 + kind, (T, N, H, D))
+        L.loopvq_residual_encode(desc, kind, x, N, N * H * D, H * D, D, codes, params, 0, N)
+        bufs.append((codes, params))
+        del x
+    ctx = torch.tensor([N], dtype=torch.int32, device="cuda")
+    off = torch.zeros(1, dtype=torch.int64, device="cuda")
+    q = synth.device_normal(30, (1, H, D))
+    out = torch.zeros((1, H, D), dtype=torch.float32, device="cuda")
+    ws = torch.zeros(L.loopvq_residual_decode_workspace_bytes(desc, 1, N), dtype=torch.uint8, device="cuda")
+    for t in range(T):
+        L.loopvq_residual_decode_attn(desc, 1, N, ctx, off, N, bufs[0][0], bufs[0][1], bufs[1][0], bufs[1][1], q, t,
+                                      D ** -0.5, out, None, ws)
+    torch.cuda.synchronize()
+    print("residual decode status", L.loopvq_read_device_status(ws))
+
+
 def _page():
     T, H, P, D, tc, G = 4, 16, 320, 128, 4, 16
     win = synth.device_normal(3, (T, H, P, D))
@@ -118,6 +144,7 @@ CASES = {
     "encode": lambda: _encode(torch.bfloat16),
     "encode-f32": lambda: _encode(torch.float32),
     "page": _page,
+    "residual": _residual,
 }
 
 

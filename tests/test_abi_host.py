@@ -207,3 +207,32 @@ def test_decode_steps_rejects_bad_step_ranges():
     assert call(2, 3) == L.LOOPVQ_ERR_INVALID_ARG
     assert call(-1, 2) == L.LOOPVQ_ERR_INVALID_ARG
     assert call(1, 2, wsb=256) == L.LOOPVQ_ERR_WORKSPACE_TOO_SMALL
+
+
+def test_residual_sizes_and_argument_errors():
+    import ctypes
+    d = L.make_residual_desc(4, 2, 128, n_heads_q=4)
+    D = ctypes.byref(d)
+    assert L.loopvq_residual_codes_bytes(d, 64) == 4 * 2 * 64 * 64
+    assert L.loopvq_residual_params_bytes(d, L.LOOPVQ_KEYS, 64) == 4 * 2 * 2 * 128 * 4
+    assert L.loopvq_residual_params_bytes(d, L.LOOPVQ_VALUES, 64) == 4 * 2 * 64 * 4 * 4
+    assert L.loopvq_residual_codes_bytes(d, 48) == 0
+    bad = L.make_residual_desc(4, 2, 96)
+    assert L._lib.loopvq_residual_codes_bytes(ctypes.byref(bad), 64) == 0
+    enc = L._lib.loopvq_residual_encode
+    assert enc(D, 0, FAKE, 0, 10, 1, 1, 1, FAKE, FAKE, 16, 64, None) == L.LOOPVQ_ERR_INVALID_ARG   # unaligned offset
+    assert enc(D, 0, FAKE, 0, 40, 1, 1, 1, FAKE, FAKE, 32, 64, None) == L.LOOPVQ_ERR_INVALID_ARG   # past pool end
+    assert enc(D, 2, FAKE, 0, 10, 1, 1, 1, FAKE, FAKE, 0, 64, None) == L.LOOPVQ_ERR_INVALID_ARG    # bad kind
+    assert enc(ctypes.byref(bad), 0, FAKE, 0, 10, 1, 1, 1, FAKE, FAKE, 0, 64, None) == L.LOOPVQ_ERR_UNSUPPORTED
+    assert enc(D, 0, FAKE, 0, 0, 1, 1, 1, FAKE, FAKE, 0, 64, None) == L.LOOPVQ_OK                 # empty
+    dec = L._lib.loopvq_residual_decode_attn
+    ws = L.loopvq_residual_decode_workspace_bytes(d, 2, 1000)
+    assert ws > 0
+
+    def call(t=0, q=FAKE, wsb=ws, pool=64):
+        return dec(D, 2, 1000, FAKE, FAKE, pool, FAKE, FAKE, FAKE, FAKE, q, L.LOOPVQ_BF16, t, 0.088, FAKE, None, FAKE,
+                   wsb, None)
+    assert call(t=4) == L.LOOPVQ_ERR_INVALID_ARG
+    assert call(q=None) == L.LOOPVQ_ERR_INVALID_ARG
+    assert call(pool=40) == L.LOOPVQ_ERR_INVALID_ARG
+    assert call(wsb=256) == L.LOOPVQ_ERR_WORKSPACE_TOO_SMALL
