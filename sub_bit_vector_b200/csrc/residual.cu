@@ -20,10 +20,11 @@
 //   key params    [T][H][pool_tokens/32][D] half2 (min, scale)
 //   value params  [T][H][pool_tokens][D/32] half2 (min, scale)
 //
-// Decode at loop step t reconstructs each token's key and value rows from
-// the t+1 residual planes (added in step order, as the encoder did; eight
-// lanes per token, each with D/8 channels) and runs split-K attention with an
-// fp32 online softmax; the last split of a (request, head) merges the splits.
+// Decode at loop step t streams tiles of the t+1 residual planes into shared
+// memory by bulk copies, rebuilds each token's key and value rows from them
+// (added in step order, as the encoder did; eight lanes per token, each with
+// D/8 channels) and runs split-K attention with an fp32 online softmax; the
+// last split of a (request, head) merges the splits.
 
 #include <cuda_fp16.h>
 #include <math.h>
@@ -152,11 +153,26 @@ __global__ void __launch_bounds__(256) res_encode_values(const ResEncParams p) {
 }
 
 // ------------------------------------------------------------------ decode
-constexpr int kRW = 16;                 // warps per CTA
-constexpr int kRThreads = kRW * 32;
+// One CTA per (split, query head, request): a producer warp streams tiles of
+// 64 tokens -- for every plane s <= t the tile's key codes, value codes, value
+// parameters and key parameters -- with bulk copies (no multicast) into a
+// ring of shared-memory stages; 16 consumer warps take one token per group of
+// eight lanes (lane i of a group owns channels i*D/8 ..), rebuild the rows
+// from the staged planes in step order and keep an fp32 online softmax.
+constexpr int kRW = 16;                       // consumer warps
+constexpr int kRThreads = (kRW + 1) * 32;     // + the producer warp
+constexpr int kRLanesPerTok = 8;
+constexpr int kRTokPerWarp = 32 / kRLanesPerTok;
+constexpr int kRTile = kRW * kRTokPerWarp;    // 64 tokens per stage
+constexpr int kRMaxStages = 4;
+constexpr int kRSmemBudget = 192 * 1024;
+
+// bytes of one plane of one tile: key codes, value codes (64 x D/2 each),
+// value parameters (64 x D/32 pairs), key parameters (2 groups x D pairs)
+__host__ __device__ inline int res_plane_bytes(int D) { return 64 * D + 8 * D + 8 * D; }
 
 struct ResDecParams {
-  int T, H, Hq, D, loop_step, max_ctx, split_len, max_splits;
+  int T, H, Hq, D, loop_step, max_ctx, split_len, max_splits, n_stages;
   const int32_t* ctx_len;
   const int64_t* tok_off;
   int64_t pool;
@@ -174,59 +190,19 @@ struct ResDecParams {
   float* partials;
 };
 
-// Eight lanes share a token (lane group g = lane / 8 of a warp takes token
-// base + g): lane i of the group owns channels i*CPL .. i*CPL+CPL-1, so one
-// lane reads CPL/2 bytes of codes per plane, its CPL key (min, scale) pairs
-// (shared by the 32 tokens of a key group: L1 hits) and one value pair.
-constexpr int kRLanesPerTok = 8;
-constexpr int kRTokPerWarp = 32 / kRLanesPerTok;
-
-template <int CPL>
-__device__ __forceinline__ void res_row(const ResDecParams& p, int h, int64_t pos, int li, float (&k)[CPL],
-                                        float (&v)[CPL]) {
-  constexpr int D = CPL * kRLanesPerTok;
-#pragma unroll
-  for (int i = 0; i < CPL; ++i) k[i] = v[i] = 0.f;
-#pragma unroll 4
-  for (int s = 0; s <= p.loop_step; ++s) {   // unrolled so that the planes' loads issue together
-    const int64_t plane = (int64_t)s * p.H + h;
-    const int64_t row = (plane * p.pool + pos) * (D / 2) + li * (CPL / 2);
-    uint32_t kc[CPL / 8], vc[CPL / 8];
-    if constexpr (CPL == 16) {
-      const uint2 a = __ldg(reinterpret_cast<const uint2*>(p.ck + row));
-      const uint2 b = __ldg(reinterpret_cast<const uint2*>(p.cv + row));
-      kc[0] = a.x; kc[1] = a.y; vc[0] = b.x; vc[1] = b.y;
-    } else {
-      kc[0] = __ldg(reinterpret_cast<const uint32_t*>(p.ck + row));
-      vc[0] = __ldg(reinterpret_cast<const uint32_t*>(p.cv + row));
-    }
-    const uint4* kp = reinterpret_cast<const uint4*>(p.pk + (plane * (p.pool / kRG) + pos / kRG) * D + li * CPL);
-    const float2 vpar = __half22float2(__ldg(p.pv + (plane * p.pool + pos) * (D / kRG) + (li * CPL) / kRG));
-#pragma unroll
-    for (int w = 0; w < CPL / 4; ++w) {
-      const uint4 pw = __ldg(kp + w);   // 4 (min, scale) pairs
-      const uint32_t pr[4] = {pw.x, pw.y, pw.z, pw.w};
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int i = w * 4 + u;
-        const float2 kpar = __half22float2(*reinterpret_cast<const __half2*>(&pr[u]));
-        const uint32_t ck = (kc[i >> 3] >> (4 * (i & 7))) & 15u;
-        const uint32_t cv = (vc[i >> 3] >> (4 * (i & 7))) & 15u;
-        k[i] = __fadd_rn(k[i], dq4(ck, kpar.x, kpar.y));
-        v[i] = __fadd_rn(v[i], dq4(cv, vpar.x, vpar.y));
-      }
-    }
-  }
-}
+struct ResConsumerSync {
+  __device__ __forceinline__ void operator()() const { asm volatile("bar.sync 1, %0;" ::"n"(kRW * 32) : "memory"); }
+};
 
 template <int CPL>
 __global__ void __launch_bounds__(kRThreads) res_decode_kernel(const ResDecParams p) {
   constexpr int D = CPL * kRLanesPerTok;
+  extern __shared__ __align__(128) uint8_t rsm[];
   __shared__ float wpart[kRW][D + 2];
-  __shared__ float csm[2 * kMaxCombineSplits + kRThreads];
+  __shared__ float csm[2 * kMaxCombineSplits + kRW * 32];
+  __shared__ __align__(8) uint64_t bars[2 * kRMaxStages];
   __shared__ int flag;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int grp = lane / kRLanesPerTok, li = lane % kRLanesPerTok;
   const int split = blockIdx.x, hq = blockIdx.y, r = blockIdx.z;
   const int h = hq / (p.Hq / p.H);
   const size_t unit = (size_t)r * p.Hq + hq;
@@ -249,9 +225,58 @@ __global__ void __launch_bounds__(kRThreads) res_decode_kernel(const ResDecParam
     return;
   }
   if (split >= n_splits) return;
-  const int t0 = split * p.split_len;
+  const int t0 = split * p.split_len;  // a multiple of 64: tiles start on key-group boundaries
   const int t1 = min(ctx, t0 + p.split_len);
+  const int n_tiles = (t1 - t0 + kRTile - 1) / kRTile;
+  const int planes = p.loop_step + 1;
+  const int pb = res_plane_bytes(D);
+  const int stage_bytes = planes * pb;
+  const int NS = p.n_stages;
+  uint64_t* full = bars;
+  uint64_t* empty = bars + kRMaxStages;
+  if (tid == 0) {
+    for (int i = 0; i < NS; ++i) {
+      mbar_init(smem_u32(full + i), 1);
+      mbar_init(smem_u32(empty + i), kRW);
+    }
+    fence_mbar_init();
+  }
+  __syncthreads();
 
+  if (warp == kRW) {  // producer
+    if (lane == 0) {
+      for (int i = 0; i < n_tiles; ++i) {
+        const int st = i % NS;
+        if (i >= NS && !mbar_wait_bounded(smem_u32(empty + st), ((i / NS) - 1) & 1)) {
+          set_fault(p.status, LOOPVQ_FAULT_TIMEOUT);
+          break;
+        }
+        const int a = t0 + i * kRTile;
+        const int n = min(kRTile, t1 - a);
+        const int ng = (n + kRG - 1) / kRG;        // key groups of the tile (1 or 2)
+        const int nr = ng * kRG;                   // rows copied: whole groups, inside the pool
+        const int64_t pos0 = off + a;
+        const uint32_t bk = 32 * D, bvp = 8 * D, bkp = 8 * D;   // offsets inside a plane block
+        const uint32_t bytes = (uint32_t)planes * (2u * nr * (D / 2) + nr * (D / kRG) * 4u + ng * D * 4u);
+        const uint32_t fb = smem_u32(full + st);
+        mbar_arrive_expect_tx(fb, bytes);
+        const uint32_t sbase = smem_u32(rsm) + (uint32_t)st * stage_bytes;
+        for (int s = 0; s < planes; ++s) {
+          const int64_t plane = (int64_t)s * p.H + h;
+          const uint32_t d0 = sbase + (uint32_t)s * pb;
+          bulk_g2s(d0, p.ck + (plane * p.pool + pos0) * (D / 2), nr * (D / 2), fb);
+          bulk_g2s(d0 + bk, p.cv + (plane * p.pool + pos0) * (D / 2), nr * (D / 2), fb);
+          bulk_g2s(d0 + 2 * bk, p.pv + (plane * p.pool + pos0) * (D / kRG), nr * (D / kRG) * 4, fb);
+          bulk_g2s(d0 + 2 * bk + bvp, p.pk + (plane * (p.pool / kRG) + pos0 / kRG) * D, ng * D * 4, fb);
+          (void)bkp;
+        }
+      }
+    }
+    return;
+  }
+
+  // consumers
+  const int grp = lane / kRLanesPerTok, li = lane % kRLanesPerTok;
   float qv[CPL];
 #pragma unroll
   for (int i = 0; i < CPL; ++i) {
@@ -263,23 +288,57 @@ __global__ void __launch_bounds__(kRThreads) res_decode_kernel(const ResDecParam
   float m = -INFINITY, l = 0.f, o[CPL];
 #pragma unroll
   for (int i = 0; i < CPL; ++i) o[i] = 0.f;
-  for (int base = t0 + warp * kRTokPerWarp; base < t1; base += kRW * kRTokPerWarp) {
-    const int tok = base + grp;
-    float kf[CPL], vf[CPL];
-    res_row<CPL>(p, h, off + min(tok, t1 - 1), li, kf, vf);  // past the end: a valid row, masked below
+  const int j = warp * kRTokPerWarp + grp;  // token of the tile
+  for (int i = 0; i < n_tiles; ++i) {
+    const int st = i % NS;
+    if (!mbar_wait_bounded(smem_u32(full + st), (i / NS) & 1)) set_fault(p.status, LOOPVQ_FAULT_TIMEOUT);
+    const int n = min(kRTile, t1 - (t0 + i * kRTile));
+    const uint8_t* sb = rsm + (size_t)st * stage_bytes;
+    float k[CPL], v[CPL];
+#pragma unroll
+    for (int c = 0; c < CPL; ++c) k[c] = v[c] = 0.f;
+    for (int s = 0; s < planes; ++s) {
+      const uint8_t* pl = sb + (size_t)s * pb;
+      uint32_t kc[CPL / 8], vc[CPL / 8];
+      if constexpr (CPL == 16) {
+        const uint2 ka = *reinterpret_cast<const uint2*>(pl + j * (D / 2) + li * 8);
+        const uint2 va = *reinterpret_cast<const uint2*>(pl + 32 * D + j * (D / 2) + li * 8);
+        kc[0] = ka.x; kc[1] = ka.y; vc[0] = va.x; vc[1] = va.y;
+      } else {
+        kc[0] = *reinterpret_cast<const uint32_t*>(pl + j * (D / 2) + li * 4);
+        vc[0] = *reinterpret_cast<const uint32_t*>(pl + 32 * D + j * (D / 2) + li * 4);
+      }
+      const float2 vpar =
+          __half22float2(*reinterpret_cast<const __half2*>(pl + 64 * D + (j * (D / kRG) + (li * CPL) / kRG) * 4));
+      const uint4* kp = reinterpret_cast<const uint4*>(pl + 72 * D + ((j / kRG) * D + li * CPL) * 4);
+#pragma unroll
+      for (int w = 0; w < CPL / 4; ++w) {
+        const uint4 pw = kp[w];
+        const uint32_t pr[4] = {pw.x, pw.y, pw.z, pw.w};
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int c = w * 4 + u;
+          const float2 kpar = __half22float2(*reinterpret_cast<const __half2*>(&pr[u]));
+          k[c] = __fadd_rn(k[c], dq4((kc[c >> 3] >> (4 * (c & 7))) & 15u, kpar.x, kpar.y));
+          v[c] = __fadd_rn(v[c], dq4((vc[c >> 3] >> (4 * (c & 7))) & 15u, vpar.x, vpar.y));
+        }
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(smem_u32(empty + st));  // the warp's reads of this stage are done
     float a = 0.f;
 #pragma unroll
-    for (int i = 0; i < CPL; ++i) a = fmaf(qv[i], kf[i], a);
+    for (int c = 0; c < CPL; ++c) a = fmaf(qv[c], k[c], a);
 #pragma unroll
     for (int x = kRLanesPerTok / 2; x >= 1; x >>= 1) a += __shfl_xor_sync(0xffffffffu, a, x);
-    const float sc = tok < t1 ? a : -INFINITY;
+    const float sc = j < n ? a : -INFINITY;
     const float mn = fmaxf(m, sc);
     if (mn != -INFINITY) {
       const float corr = exp2f(m - mn);
       const float pw = exp2f(sc - mn);
       l = fmaf(l, corr, pw);
 #pragma unroll
-      for (int i = 0; i < CPL; ++i) o[i] = fmaf(o[i], corr, pw * vf[i]);
+      for (int c = 0; c < CPL; ++c) o[c] = fmaf(o[c], corr, pw * v[c]);
       m = mn;
     }
   }
@@ -292,23 +351,24 @@ __global__ void __launch_bounds__(kRThreads) res_decode_kernel(const ResDecParam
     const float ca = m == -INFINITY ? 0.f : exp2f(m - mn);
     const float cb = mo == -INFINITY ? 0.f : exp2f(mo - mn);
 #pragma unroll
-    for (int i = 0; i < CPL; ++i) {
-      const float oo = __shfl_xor_sync(0xffffffffu, o[i], x);
-      o[i] = o[i] * ca + oo * cb;
+    for (int c = 0; c < CPL; ++c) {
+      const float oo = __shfl_xor_sync(0xffffffffu, o[c], x);
+      o[c] = o[c] * ca + oo * cb;
     }
     l = l * ca + lo_ * cb;
     m = mn;
   }
   if (grp == 0) {
 #pragma unroll
-    for (int i = 0; i < CPL; ++i) wpart[warp][li * CPL + i] = o[i];
+    for (int c = 0; c < CPL; ++c) wpart[warp][li * CPL + c] = o[c];
     if (li == 0) { wpart[warp][D] = m; wpart[warp][D + 1] = l; }
   }
-  __syncthreads();
+  const ResConsumerSync csync;
+  csync();
   float* part = p.partials + (unit * p.max_splits + split) * (size_t)(D + 4);
   float M = -INFINITY;
   for (int w = 0; w < kRW; ++w) M = fmaxf(M, wpart[w][D]);
-  for (int d = tid; d < D + 2; d += blockDim.x) {
+  for (int d = tid; d < D + 2; d += kRW * 32) {
     float acc = 0.f;
     if (d != D) {
       for (int w = 0; w < kRW; ++w) {
@@ -319,13 +379,13 @@ __global__ void __launch_bounds__(kRThreads) res_decode_kernel(const ResDecParam
     part[d] = (d == D) ? M : acc;
   }
   __threadfence();
-  __syncthreads();
+  csync();
   if (tid == 0) flag = (atomicAdd(p.tickets + unit, 1u) == (uint32_t)(n_splits - 1)) ? 1 : 0;
-  __syncthreads();
+  csync();
   if (flag) {
     __threadfence();
     combine_splits(p.partials + unit * p.max_splits * (size_t)(D + 4), n_splits, D, p.out + unit * D, 0,
-                   p.lse ? p.lse + unit : nullptr, csm, tid, kRThreads, BlockSync{});
+                   p.lse ? p.lse + unit : nullptr, csm, tid, kRW * 32, csync);
     if (tid == 0) atomicExch(p.tickets + unit, 0u);
   }
 }
@@ -336,7 +396,8 @@ static void res_plan(int64_t units, int max_ctx, int n_sm, int* split_len, int* 
   if (s > cap) s = cap;
   if (s < 1) s = 1;
   int len = (max_ctx + s - 1) / s;
-  if (len < 1) len = 1;
+  len = ((len + kRTile - 1) / kRTile) * kRTile;  // tiles start on key-group boundaries
+  if (len < kRTile) len = kRTile;
   *split_len = len;
   *max_splits = max_ctx > 0 ? (max_ctx + len - 1) / len : 1;
 }
@@ -419,8 +480,8 @@ extern "C" loopvq_status loopvq_residual_decode_attn(const loopvq_residual_desc*
   if (!(softmax_scale == softmax_scale)) return LOOPVQ_ERR_INVALID_ARG;
   if (!ctx_len || !tok_off || !codesK || !paramsK || !codesV || !paramsV || !q || !out || !workspace)
     return LOOPVQ_ERR_INVALID_ARG;
-  if (((uintptr_t)paramsK & 15) || ((uintptr_t)paramsV & 3) || ((uintptr_t)codesK & 7) || ((uintptr_t)codesV & 7) ||
-      ((uintptr_t)workspace & 255))
+  if (((uintptr_t)paramsK & 15) || ((uintptr_t)paramsV & 15) || ((uintptr_t)codesK & 15) ||
+      ((uintptr_t)codesV & 15) || ((uintptr_t)workspace & 255))
     return LOOPVQ_ERR_INVALID_ARG;
   if (workspace_bytes < loopvq_residual_decode_workspace_bytes(desc, batch, max_ctx_len))
     return LOOPVQ_ERR_WORKSPACE_TOO_SMALL;
@@ -441,10 +502,24 @@ extern "C" loopvq_status loopvq_residual_decode_attn(const loopvq_residual_desc*
   p.status = (uint32_t*)workspace;
   p.tickets = (uint32_t*)((uint8_t*)workspace + ws.tickets_off);
   p.partials = (float*)((uint8_t*)workspace + ws.partials_off);
+  const int stage_bytes = (loop_step + 1) * res_plane_bytes(g.D);
+  int ns = kRSmemBudget / stage_bytes;
+  if (ns > kRMaxStages) ns = kRMaxStages;
+  if (ns < 1) return LOOPVQ_ERR_UNSUPPORTED;   // more planes than one stage can hold
+  p.n_stages = ns;
+  const size_t smem = (size_t)ns * stage_bytes;
   dim3 grid(ms, g.Hq, batch);
-  if (g.D == 128)
-    res_decode_kernel<16><<<grid, kRThreads, 0, (cudaStream_t)stream>>>(p);
-  else
-    res_decode_kernel<8><<<grid, kRThreads, 0, (cudaStream_t)stream>>>(p);
+  cudaStream_t s = (cudaStream_t)stream;
+  if (g.D == 128) {
+    if (cudaFuncSetAttribute(res_decode_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+        cudaSuccess)
+      return LOOPVQ_ERR_CUDA;
+    res_decode_kernel<16><<<grid, kRThreads, smem, s>>>(p);
+  } else {
+    if (cudaFuncSetAttribute(res_decode_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+        cudaSuccess)
+      return LOOPVQ_ERR_CUDA;
+    res_decode_kernel<8><<<grid, kRThreads, smem, s>>>(p);
+  }
   return cudaGetLastError() == cudaSuccess ? LOOPVQ_OK : LOOPVQ_ERR_CUDA;
 }
