@@ -398,6 +398,65 @@ def all_steps_measurement(layers, device, reps=400):
                     f"{len(layers)} rotating layer caches"}
 
 
+def residual_measurement(device, n_layers=4, reps=40):
+    """Second workload on the same shape: adjacent-loop KV-residual 4-bit
+    coding of one layer's [4][32768][16][128] keys and values, then decode
+    attention at each loop step (every token coded, no bf16 window); rotating
+    over layer caches larger than L2."""
+    import torch
+    from sub_bit_vector_b200 import loopvq as L, synth
+    desc = L.make_residual_desc(T, H, D)
+    layers = []
+    enc_ms = None
+    for i in range(n_layers):
+        bufs = []
+        for kind in (L.LOOPVQ_KEYS, L.LOOPVQ_VALUES):
+            codes = torch.zeros(L.loopvq_residual_codes_bytes(desc, CTX), dtype=torch.uint8, device=device)
+            params = torch.zeros(L.loopvq_residual_params_bytes(desc, kind, CTX) // 2, dtype=torch.float16,
+                                 device=device)
+            x = synth.device_normal(1500 + 2 * i + kind, (T, CTX, H, D), device=device)
+            L.loopvq_residual_encode(desc, kind, x, CTX, CTX * H * D, H * D, D, codes, params, 0, CTX)
+            if i == 0 and kind == L.LOOPVQ_KEYS:
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                torch.cuda.synchronize()
+                e0.record()
+                L.loopvq_residual_encode(desc, kind, x, CTX, CTX * H * D, H * D, D, codes, params, 0, CTX)
+                e1.record()
+                torch.cuda.synchronize()
+                enc_ms = e0.elapsed_time(e1)
+            bufs.append((codes, params))
+            del x
+        ws = torch.zeros(L.loopvq_residual_decode_workspace_bytes(desc, 1, CTX), dtype=torch.uint8, device=device)
+        layers.append((bufs, ws))
+    ctx = torch.tensor([CTX], dtype=torch.int32, device=device)
+    off = torch.zeros(1, dtype=torch.int64, device=device)
+    q = synth.device_normal(1599, (1, H, D), device=device)
+    out = torch.zeros((1, H, D), dtype=torch.float32, device=device)
+    per_step = []
+    for t in range(T):
+        def run(b):
+            (ck, pk), (cv, pv) = b[0]
+            L.loopvq_residual_decode_attn(desc, 1, CTX, ctx, off, CTX, ck, pk, cv, pv, q, t, D ** -0.5, out, None,
+                                          b[1])
+        for b in layers:
+            run(b)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for i in range(reps):
+            run(layers[i % n_layers])
+        e1.record()
+        torch.cuda.synchronize()
+        us = e0.elapsed_time(e1) * 1e3 / reps
+        by = (t + 1) * H * CTX * (D // 2 * 2 + (D // 32) * 4 + D * 4 // 32) + H * D * 6
+        per_step.append({"loop_step": t, "us_per_launch": us, "algorithmic_bytes": by, "GB_per_s": by / us / 1e3,
+                         "kv_tokens_per_s": CTX / (us * 1e-6)})
+    faults = max(L.loopvq_read_device_status(b[1])[1] for b in layers)
+    return {"encode_keys_ms_per_tensor": enc_ms, "decode": per_step, "device_fault_bits": faults,
+            "what": "4-bit residuals between adjacent loop steps (fp16 min/scale per 32), decode rebuilding step t "
+                    "from t+1 planes; batch 1, 16x128, ctx 32768"}
+
+
 def encode_measurement(device, with_oracle, reps=5):
     """Loop-axis encode of a 32768-token prefill's keys [4][32768][16][128]
     bf16 at 0.5 bit (tensor-core kernel); with_oracle adds the oracle's rate
@@ -600,6 +659,12 @@ def run_gpu(args):
                    "pinned host, stream sync per step"}
 
     steps_fused = all_steps_measurement(layers, device) if not args.no_extras else None
+    residual = None
+    if not args.no_extras:
+        try:
+            residual = residual_measurement(device)
+        except Exception as exc:   # a context figure: report, never lose the line for it
+            residual = {"error": f"{type(exc).__name__}: {exc}"}
     dense = dense_comparator(device) if not args.no_extras else None
     sdpa = sdpa_comparator(device) if not args.no_extras else None
     enc = (encode_measurement(device, with_oracle=(rank == 0 and world == 1 and not args.no_cpu_baseline))
@@ -611,7 +676,7 @@ def run_gpu(args):
                 "scaling": "weak", "vs_baseline": None, "dtype": "u8 codes, f32 accumulate", "data": "synthetic",
                 "config": dict(_config(), parallelism=f"replicas x{world}" if world > 1 else "single GPU"),
                 "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches,
-                "clocks": clocks, "all_steps_one_launch": steps_fused, "dense_bf16_comparator": dense, "torch_sdpa_bf16": sdpa, "encode": enc,
+                "clocks": clocks, "all_steps_one_launch": steps_fused, "kv_residual_4bit": residual, "dense_bf16_comparator": dense, "torch_sdpa_bf16": sdpa, "encode": enc,
                 "device_fault_bits": max(status)}
         print(json.dumps(line), flush=True)
     del decode_graphs, encode_graphs
