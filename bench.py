@@ -6,9 +6,9 @@ Workload: Ouro-1.4B-shaped decode attention of one layer -- batch 1, 16 KV
 heads x head_dim 128, 4 loop steps, Tc = 4, context 32768 tokens, 0.5 bit
 (256-entry codebooks over 4 channels x 4 steps), first 64 and last 256 tokens
 in bf16.  One step = one generated token through that layer: the four loop
-steps' decode-attention launches, plus (every 8th step, as the serving rule
-on the LoopVQ project page encodes the oldest recent page after every 8
-generated tokens) the page encode of 8 tokens for K and V.  Eight distinct
+steps' decode-attention launches, plus, every 8th step, the 8-token page
+encode of K and V (in the serving scheme of the LoopVQ project page, one page
+leaves the bf16 recent window and is coded for each 8 new tokens).  Eight distinct
 layer caches (~350 MB) rotate across steps so no launch reads warm L2.
 
 Metric: KV tokens/s = (context tokens x loop steps attended) / time.  The

@@ -8,12 +8,12 @@
  *     vector quantization": one codebook index covers G/Tc channels of each
  *     of Tc consecutive loop steps; at inference each loop step reads the
  *     shared index through its own slice of the codebook.
- *   - "Serving in SGLang": new keys/values are written in bf16; the first
- *     n_sink and the most recent n_recent tokens stay bf16 at every loop step
- *     ("Write in bf16"); after every 8 generated tokens the oldest recent page
- *     is encoded ("Encode in pages"); at loop step t the attention kernel reads
- *     keys and values from the indices through slice B_t and merges the result
- *     with the bf16 attention ("Attend from indices").
+ *   - "Serving in SGLang": a new token's keys/values enter the cache in bf16,
+ *     and the n_sink sink tokens and the n_recent recent ones are kept in bf16
+ *     for every loop step ("Write in bf16"); for each 8 new tokens the page
+ *     leaving the recent window is coded ("Encode in pages"); at step t the
+ *     attention reads the coded body through slice B_t and combines it with
+ *     the bf16 part ("Attend from indices").
  *   - "Results -- Long-context retrieval": n_sink = 64, n_recent = 256.
  *
  * Notation: T loop steps, Tc steps per code, NB = T/Tc code blocks,

@@ -13,11 +13,11 @@ Sources (all from the LoopVQ web pages):
 * Same page, "Component 1 -- Loop-axis vector quantization": one index
   covers channels of several *consecutive* loop steps.
 * Same page, "Serving in SGLang" -- "Write in bf16", "Encode in pages",
-  "Attend from indices": new K/V are written in bf16; the first n_sink and
-  most recent n_recent tokens stay bf16 at every loop step; after every 8
-  generated tokens the oldest recent page is encoded; at loop step t the
-  kernel reads keys/values from the indices through slice B_t and merges with
-  the bf16 attention.
+  "Attend from indices": a new token's K/V enter the cache in bf16; the sink
+  tokens and the recent window are kept in bf16 for every loop step; for
+  each 8 new tokens, the page leaving the recent window is coded; at step t
+  the attention reads the coded body through slice B_t and combines it with
+  the bf16 part.
 * Same page, "Results -- Long-context retrieval": n_sink = 64 and
   n_recent = 256.
 * Same page, "Highlights" and "Efficiency": 0.5 / 0.25 bit per element is
@@ -240,9 +240,9 @@ def dequantize(idx: np.ndarray, codebook: np.ndarray, loop_step: int, tc: int) -
 def window_split(ctx_len: int, n_sink: int, n_recent: int, page: int):
     """Split a context of ``ctx_len`` tokens into (sink, body, recent) counts.
 
-    Project page, "Serving in SGLang": the first n_sink and the most recent
-    n_recent tokens stay bf16 at every loop step, and after every 8 generated
-    tokens the oldest recent page is encoded.  Read as: the recent window
+    Project page, "Serving in SGLang": the sink tokens and the recent window
+    are kept in bf16 for every loop step, and for each 8 new tokens the page
+    leaving the recent window is coded.  Read as: the recent window
     holds n_recent .. n_recent+page-1 tokens, so the encoded body is whole
     pages; a context no longer than n_sink + n_recent is all bf16.  The
     current token is counted in ``ctx_len`` and sits in the recent window.
@@ -494,10 +494,10 @@ def attention_mse_codebook_grad(q, loop_step, tc, idx_k, idx_v, codebook_k, code
 # second workload: adjacent-loop KV-residual quantization (4-bit)
 # --------------------------------------------------------------------------
 # FlashLoop page (thelatestinai.com, "Figure 2 (c)", "Figure 3 (c-d)", "Table
-# 2", "Figure 4"): K/V residuals between adjacent loop steps shrink with loop
-# depth, and recursively quantizing adjacent-loop residuals gives a lower
-# reconstruction error than quantizing every loop's complete K/V; the method
-# uses 4-bit residuals along the axes of per-loop KIVI4.  Readings where the
+# 2", "Figure 4"): the change of K/V from one loop step to the next gets
+# smaller deeper in the loop, so coding each step as a residual over the
+# previous step loses less than coding each step's K/V on its own; the page
+# codes these residuals with 4 bits, on the axes KIVI's 4-bit quantizer uses.  Readings where the
 # page is silent: KIVI's quantizer (asymmetric, 16 levels, min and scale per
 # group of 32; keys grouped per channel over 32 consecutive tokens, values
 # per token over 32 consecutive channels; min and scale stored in fp16);

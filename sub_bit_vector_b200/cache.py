@@ -163,10 +163,10 @@ class DecodeCache:
 class PagedCache:
     """Incremental serving cache of one layer (K and V) for a batch of requests.
 
-    LoopVQ project page, "Serving in SGLang": new keys and values are written
-    in bf16; the first ``n_sink`` and the most recent tokens stay bf16; after
-    every ``page`` generated tokens the oldest recent page is encoded; decode
-    reads the body from the indices.  Here the body lives in fixed-size pages
+    LoopVQ project page, "Serving in SGLang": a new token's keys and values
+    enter the cache in bf16; the ``n_sink`` sink tokens and the recent window
+    are kept in bf16; for each ``page`` new tokens the page leaving the recent
+    window is coded; decode reads the coded body from the indices.  Here the body lives in fixed-size pages
     of the index pools (``body_page_tokens`` tokens each, taken from a free
     list, listed per request in a page table) and the recent tokens in a ring
     of ``n_recent + page`` slots per request, so nothing is ever moved.

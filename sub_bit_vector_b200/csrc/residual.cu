@@ -1,10 +1,10 @@
 // Adjacent-loop KV-residual 4-bit quantization and decode attention (sm_100a).
 //
 // FlashLoop page (thelatestinai.com; "Figure 2 (c)", "Figure 3 (c-d)",
-// "Table 2", "Figure 4"): K/V residuals between adjacent loop steps shrink
-// with depth, and recursively quantizing them reconstructs the cache better
-// than quantizing every loop's complete K/V; the method uses 4-bit residuals
-// along the axes of per-loop KIVI4.  Step 0 codes K_0; step t codes
+// "Table 2", "Figure 4"): the change of K/V from one loop step to the next
+// gets smaller deeper in the loop, so coding each step as a residual over the
+// previous step loses less than coding each step's K/V on its own; the page
+// codes these residuals with 4 bits, on the axes KIVI's 4-bit quantizer uses.  Step 0 codes K_0; step t codes
 // R_t = K_t - Khat_{t-1}, the residual against the previous reconstruction,
 // and Khat_t = Khat_{t-1} + Q(R_t).  Q is KIVI's quantizer: 16 levels, an
 // fp16 minimum and an fp16 scale per group of 32 values; keys are grouped

@@ -557,9 +557,10 @@ def test_residual_reconstruction_telescopes():
 
 
 def test_residual_coding_beats_per_step_coding_on_loop_correlated_data():
-    """FlashLoop page, Figure 2 (c): recursively coding adjacent-loop residuals
-    reconstructs a loop-correlated cache with lower error than coding every
-    loop step's K/V on its own at the same bits."""
+    """FlashLoop page, Figure 2 (c): coding each step as a residual over the
+    previous step's reconstruction reconstructs a loop-correlated cache with
+    lower error than coding every loop step's K/V on its own at the same
+    bits."""
     X = synth.loop_correlated(seed=720, n_loop=4, n_tokens=96, n_heads=2, head_dim=64, rho=0.95)
     for kind in ("k", "v"):
         _, _, _, recon = O.residual_encode(X, kind)
