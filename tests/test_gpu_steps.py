@@ -118,3 +118,57 @@ def test_new_token_per_step_is_used_and_stored():
     for t in range(4):
         for r in range(2):
             assert torch.equal(c.winK[t, :, last[r]], nk[t, r]) and torch.equal(c.winV[t, :, last[r]], nv[t, r])
+
+
+def test_steps_launch_over_paged_body_and_ring_window():
+    """All four steps in one launch over a paged body (shuffled 256-token
+    pages) and ring windows that wrap: every step matches the oracle."""
+    L = _L()
+    case = Case(seed=34, ctx_lens=[5000, 700, 333], H=2, Hq=4)
+    c = case.c
+    rng = np.random.default_rng(35)
+    bpt, ns, nr, pg = 256, 64, 256, 8
+    ring = nr + pg
+    B = len(c.ctx_lens)
+    max_pages = -(-max(c.splits[r][1] for r in range(B)) // bpt)
+    n_phys = B * max_pages + 3
+    perm = rng.permutation(n_phys)
+    idxK = torch.zeros(L.loopvq_index_pool_bytes(c.desc, n_phys * bpt), dtype=torch.uint8, device="cuda")
+    idxV = torch.zeros_like(idxK)
+    pages = np.full((B, max_pages), -1, dtype=np.int32)
+    heads = np.array([200, 8, 0], dtype=np.int32)
+    stride = ns + ring
+    winK = torch.zeros((c.T, c.H, B * stride, c.D), dtype=torch.bfloat16, device="cuda")
+    winV = torch.zeros_like(winK)
+    nxt = 0
+    for r in range(B):
+        s, body, rec = c.splits[r]
+        wk, wv, ck, cv = case.req[r]
+        for pi in range(-(-body // bpt)):
+            pages[r, pi] = perm[nxt]
+            nxt += 1
+            n = min(bpt, body - pi * bpt)
+            for kind, src, pool in ((0, ck, idxK), (1, cv, idxV)):
+                t = torch.from_numpy(np.ascontiguousarray(src[:, :, pi * bpt:pi * bpt + n])).cuda()
+                L.loopvq_index_pool_pack(c.desc, kind, t, n, pool, int(pages[r, pi]) * bpt, n_phys * bpt)
+        for i in range(s + rec):
+            row = r * stride + (i if i < s else ns + (heads[r] + i - s) % ring)
+            winK[:, :, row] = torch.from_numpy(np.ascontiguousarray(wk[:, :, i], dtype=np.float32)).cuda().to(
+                torch.bfloat16)
+            winV[:, :, row] = torch.from_numpy(np.ascontiguousarray(wv[:, :, i], dtype=np.float32)).cuda().to(
+                torch.bfloat16)
+    assert heads[0] + c.splits[0][2] > ring   # request 0's ring wraps
+    pages_dev = torch.from_numpy(pages).cuda()
+    heads_dev = torch.from_numpy(heads).cuda()
+    win_off = torch.arange(B, dtype=torch.int64, device="cuda") * stride
+    lay = L.make_layout(B, ns, nr, pg, c.max_ctx_len, c.ctx_dev, c.body_off_dev, win_off, n_phys * bpt, B * stride,
+                        L.LOOPVQ_LAYOUT_PAGED_BODY | L.LOOPVQ_LAYOUT_RING_WINDOW, pages_dev, bpt, max_pages,
+                        heads_dev, ring)
+    q = torch.from_numpy(np.ascontiguousarray(case.q, dtype=np.float32)).cuda().to(torch.bfloat16)
+    out = torch.zeros((4, B, c.Hq, c.D), dtype=torch.float32, device="cuda")
+    lse = torch.zeros((4, B, c.Hq), dtype=torch.float32, device="cuda")
+    ws = torch.zeros(L.loopvq_decode_steps_workspace_bytes(c.desc, lay, 4), dtype=torch.uint8, device="cuda")
+    L.loopvq_decode_attn_steps(c.desc, c.cbK, c.cbV, lay, idxK, idxV, winK, winV, q, 0, 4, c.D ** -0.5, out, lse, ws)
+    torch.cuda.synchronize()
+    assert L.loopvq_read_device_status(ws)[1] == 0
+    _check(case, 0, 4, out.cpu().numpy(), lse.cpu().numpy())
