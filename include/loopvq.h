@@ -24,9 +24,11 @@
  * Conventions for every entry point:
  *   - The caller owns all memory.  Pointers documented "device" must be
  *     device (or managed) memory of the current CUDA device; "host" pointers
- *     are ordinary host memory.  The library allocates nothing and keeps no
- *     global mutable state; calls on different streams are independent unless
- *     they share output or workspace buffers.
+ *     are ordinary host memory.  The library allocates nothing.  Its only
+ *     global state is the device word of encode faults
+ *     (loopvq_read_encode_faults) and the fixed scratch array of
+ *     loopvq_decode_attn_noalloc; otherwise calls on different streams are
+ *     independent unless they share output or workspace buffers.
  *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy
  *     default stream).  Argument errors are detected on the host and returned
  *     before anything is launched.
