@@ -406,6 +406,33 @@ def test_kmeans_update_is_the_distortion_minimiser_and_a_fixed_point():
     np.testing.assert_allclose(again, new, rtol=0, atol=1e-13)
 
 
+def test_distortion_hand_value_and_element_identity():
+    """The distortion is the sum, over every sub-vector, of its squared
+    distance to its codeword: 1 on the hand-worked fixture (one element off by
+    one), the encoder's best distances summed, and -- every element lying in
+    exactly one sub-vector -- the mean squared reconstruction error times the
+    element count, with several code blocks, heads and slots."""
+    g = _load("hand_worked.json")
+    X = np.array(g["X_T_N_H_D"], dtype=np.float64)
+    cb = np.array(g["codebook_NB_H_J_C_Tc_W"], dtype=np.float64)
+    idx = np.array(g["idx_NB_H_N_J"])
+    assert O.distortion(X, idx, cb, g["geometry"]["Tc"]) == 1.0
+    rng = np.random.default_rng(760)
+    T, tc, N, H, D, G, C = 4, 2, 37, 3, 16, 4, 9     # NB = 2 blocks, W = 2, J = 8
+    X = rng.standard_normal((T, N, H, D))
+    cb = rng.standard_normal((T // tc, H, D // (G // tc), C, tc, G // tc))
+    idx, d1, _ = O.encode(X, cb, tc)
+    total = O.distortion(X, idx, cb, tc)
+    assert total == pytest.approx(float(np.sum(d1)), rel=1e-12)
+    assert total == pytest.approx(O.reconstruction_mse(X, idx, cb, tc) * X.size, rel=1e-12)
+    # a code that is not the nearest one adds exactly its extra distance
+    idx2 = idx.copy()
+    idx2[1, 2, 5, 3] = (idx[1, 2, 5, 3] + 1) % C
+    sub = X[2:4, 5, 2, 6:8].reshape(-1)   # block 1, token 5, head 2, slot 3: channels 6..7 of steps 2..3, order [t][w]
+    extra = np.sum((sub - cb[1, 2, 3, idx2[1, 2, 5, 3]].reshape(-1)) ** 2) - d1[1, 2, 5, 3]
+    assert O.distortion(X, idx2, cb, tc) == pytest.approx(total + extra, rel=1e-12)
+
+
 def test_lloyd_distortion_never_increases():
     X = _small_kv(530)
     cb = synth.codebook_from_rows(X, 4, 16, 32, seed=531)
@@ -535,6 +562,73 @@ def test_quantize4_error_bound_and_constant_group():
         assert q.max() <= 15
     q, l, c = O.quantize4_group(np.full(32, 0.3, dtype=np.float32))
     assert c == 0 and not q.any() and np.all(O.dequantize4(q, l, c) == np.float32(np.float16(0.3)))
+
+
+def _residual_hand_worked_inputs(g, kind):
+    """The fixture's inputs and hand-derived expectations (closed forms stated
+    in tests/golden/residual_hand_worked.json)."""
+    T, N, H, D = g["shape_T_N_H_D"]
+    n = np.arange(N)[:, None]
+    d = np.arange(D)[None, :]
+    delta = g["delta"]
+    if kind == "k":
+        x0 = 0.5 * (n % 16) + 8.0 * (d % 2) + delta * (n == 5)
+        code0 = np.broadcast_to(n % 16, (N, D))
+        hat0 = 0.5 * (n % 16) + 8.0 * (d % 2)
+    else:
+        x0 = 0.5 * (d % 16) + 8.0 * (n % 2) + delta * (d == 5)
+        code0 = np.broadcast_to(d % 16, (N, D))
+        hat0 = 0.5 * (d % 16) + 8.0 * (n % 2)
+    code1 = (n + d) % 16
+    x1 = hat0 + 0.25 * code1
+    X = np.stack([x0, x1])[:, :, None, :].astype(np.float32)      # [T][N][H][D]
+    return X, code0, hat0, code1, x1
+
+
+@pytest.mark.parametrize("kind", ["k", "v"])
+def test_residual_hand_worked_two_steps(kind):
+    """FlashLoop page, Figure 2 (c) and Figure 3 (c-d), with the readings of
+    KIVI's axes and the reconstruction as the residual's reference: a
+    two-step case derived by hand.  Coding step 1 against K_0 instead of
+    Khat_0, or grouping along the other axis, changes the codes or the
+    parameters checked here."""
+    g = _load("residual_hand_worked.json")
+    X, code0, hat0, code1, x1 = _residual_hand_worked_inputs(g, kind)
+    codes, lo, sc, recon = O.residual_encode(X, kind)
+    np.testing.assert_array_equal(codes[0, 0], code0)
+    np.testing.assert_array_equal(codes[1, 0], code1)
+    np.testing.assert_array_equal(recon[0, :, 0], hat0.astype(np.float32))
+    np.testing.assert_array_equal(recon[1, :, 0], x1.astype(np.float32))
+    e = g["keys" if kind == "k" else "values"]
+    par = np.arange(32) % 2
+    if kind == "k":     # one token group: lo/scale [T][H][1][D]
+        np.testing.assert_array_equal(lo[0, 0, 0], np.array(e["step0"]["lo_per_channel_parity"])[par])
+        assert lo.shape == (2, 1, 1, 32)
+    else:               # one channel group per token: [T][H][N][1]
+        np.testing.assert_array_equal(lo[0, 0, :, 0], np.array(e["step0"]["lo_per_token_parity"])[par])
+        assert lo.shape == (2, 1, 32, 1)
+    assert np.all(sc[0] == np.float16(e["step0"]["scale"])) and np.all(sc[1] == np.float16(e["step1"]["scale"]))
+    assert np.all(lo[1] == np.float16(e["step1"]["lo"]))
+    for sp in e["spot"]:
+        t, n_, d_ = sp["t"], sp["n"], sp["d"]
+        assert X[t, n_, 0, d_] == sp["x"]
+        assert codes[t, 0, n_, d_] == sp["code"]
+        assert recon[t, n_, 0, d_] == sp["recon"]
+        assert O.residual_reconstruct(codes, lo, sc, kind, t)[n_, 0, d_] == sp["recon"]
+
+
+def test_residual_hand_worked_rejects_the_other_readings():
+    """The fixture tells the readings apart: against the raw previous step
+    the key residual of channel 11 has its minimum at -delta; grouped along
+    the other axis the step-0 scale is fp16(8/15), not 0.5."""
+    g = _load("residual_hand_worked.json")
+    X, _, _, _, _ = _residual_hand_worked_inputs(g, "k")
+    raw_resid = X[1, :, 0, 11] - X[0, :, 0, 11]
+    _, lo_raw, _ = O.quantize4_group(raw_resid)
+    assert lo_raw == np.float16(-g["delta"])
+    # keys grouped per token (the values' axis): token 0 over channels
+    _, _, sc_swapped = O.quantize4_group(X[0, 0, 0, :])
+    assert sc_swapped == np.float16(8.0 / 15.0) == np.float16(0.533203125)
 
 
 def test_residual_reconstruction_telescopes():
