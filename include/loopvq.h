@@ -25,17 +25,17 @@
  *   - The caller owns all memory.  Pointers documented "device" must be
  *     device (or managed) memory of the current CUDA device; "host" pointers
  *     are ordinary host memory.  The library allocates nothing.  Its only
- *     global state is the device word of encode faults
- *     (loopvq_read_encode_faults) and the fixed scratch array of
- *     loopvq_decode_attn_noalloc; otherwise calls on different streams are
- *     independent unless they share output or workspace buffers.
+ *     global state is the fixed scratch array of loopvq_decode_attn_noalloc;
+ *     otherwise calls on different streams are independent unless they share
+ *     output, workspace or fault-word buffers.
  *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy
  *     default stream).  Argument errors are detected on the host and returned
  *     before anything is launched.
  *   - Faults that only the device can see (a code >= n_codes, a context or
- *     offset outside the pools) never trap: the kernel sets a bit in the
- *     workspace's status word, skips the offending work and finishes; read it
- *     with loopvq_read_device_status().
+ *     offset outside the pools, a bounded wait that gave up) never trap: the
+ *     kernel ORs a LOOPVQ_FAULT_* bit into a word in caller memory -- the
+ *     workspace's status word (loopvq_read_device_status) or a fault_bits
+ *     argument -- skips the offending work and finishes.
  *   - All integer sizes are element counts unless a name ends in _bytes.
  */
 #ifndef LOOPVQ_H_
@@ -97,11 +97,14 @@ typedef struct {
 /*
  * Layout flag: the caller guarantees that no kernel that may still be running
  * when the decode kernel starts writes the layout arrays (ctx_len, body_off,
- * win_off), the index pools or the codebooks.  The decode kernel is always
- * launched as a programmatic dependent of the previous kernel in the stream;
- * with this flag it starts streaming index tiles before that kernel has
- * finished (queries, windows, outputs and the workspace are still touched
- * only after it has).  Without the flag nothing is read before then.
+ * win_off, body_pages, win_head), the index pools or the codebooks.  The
+ * decode kernel is always launched as a programmatic dependent of the
+ * previous kernel in the stream; with this flag it starts streaming index
+ * tiles before that kernel has finished.  Queries, window pools, new-token
+ * rows, outputs and the workspace are touched only after it has, with or
+ * without the flag (an earlier decode call of the same cache may still be
+ * storing its new token into the window pool).  Without the flag nothing is
+ * read before then.
  */
 #define LOOPVQ_LAYOUT_STATIC_INPUTS 0x1u
 /* The body lives in pages of the index pool listed by body_pages (see below)
@@ -110,10 +113,6 @@ typedef struct {
 /* The recent tokens live in a ring of win_ring slots per request (see below)
  * instead of right after the sink tokens. */
 #define LOOPVQ_LAYOUT_RING_WINDOW 0x4u
-/* With LOOPVQ_LAYOUT_STATIC_INPUTS: the window pools are not written by the
- * kernel that precedes the call either (true when the current token arrives
- * through new_k/new_v), so the window rows are streamed early too. */
-#define LOOPVQ_LAYOUT_STATIC_WINDOWS 0x8u
 
 /*
  * Cache layout of one decode batch.  Request r has ctx_len[r] tokens, the
@@ -155,9 +154,10 @@ typedef struct {
   int32_t win_ring;           /* >= n_recent + page - 1 */
   int32_t reserved;           /* 0 */
   /* The current token's key and value at this loop step, device bf16
-   * [batch][n_heads_kv][head_dim], or NULL.  When set, the decode uses them
-   * for the current token (the last window token) and also stores them in
-   * its window slot -- the pages' "write in bf16" fused into attention. */
+   * [batch][n_heads_kv][head_dim], 8-byte aligned, or NULL.  When set, the
+   * decode uses them for the current token (the last window token) and also
+   * stores them in its window slot -- the pages' "write in bf16" fused into
+   * attention. */
   const void* new_k;
   const void* new_v;
 } loopvq_cache_layout;
@@ -258,21 +258,19 @@ LOOPVQ_API loopvq_status loopvq_index_pool_unpack(const loopvq_codebook_desc* de
  * the tensor cores (tcgen05: d = |x|^2 + |c|^2 - 2 x.c in fp32, with every
  * near-tie re-solved exactly from the differences); everything else runs the
  * CUDA-core kernel.  Both return the nearest codeword up to fp32 rounding of
- * distances that are equal within it.  A device-side timeout (never expected)
- * leaves that tile's codes unwritten and sets LOOPVQ_FAULT_TIMEOUT in the
- * word read by loopvq_read_encode_faults.
+ * distances that are equal within it.
+ *   fault_bits : device uint32, 4-byte aligned, into which the kernel ORs
+ *               LOOPVQ_FAULT_* bits (the caller zeroes it and reads it after
+ *               the stream), or NULL to drop them.  The only fault is a
+ *               bounded wait on the tensor cores that gave up (never
+ *               expected): that tile's codes are left unwritten and
+ *               LOOPVQ_FAULT_TIMEOUT is set.
  */
 LOOPVQ_API loopvq_status loopvq_encode(const loopvq_codebook_desc* desc, const void* cb_packed,
                             loopvq_kind kind, const void* x, loopvq_dtype x_dtype,
                             int64_t n_tokens, int64_t stride_t, int64_t stride_n,
                             int64_t stride_h, uint8_t* idx_pool, int64_t tok_off,
-                            int64_t pool_tokens, loopvq_stream_t stream);
-
-/* Waits for `stream`, then reads the encoder's device fault word (one per
- * device, shared by all encode calls): LOOPVQ_OK if zero, else
- * LOOPVQ_ERR_DEVICE_FAULT with the LOOPVQ_FAULT_* bits in *bits (if non-NULL).
- * clear != 0 zeroes the word afterwards. */
-LOOPVQ_API loopvq_status loopvq_read_encode_faults(uint32_t* bits, int32_t clear, loopvq_stream_t stream);
+                            int64_t pool_tokens, uint32_t* fault_bits, loopvq_stream_t stream);
 
 /* ------------------------------------------------ codebook construction */
 
@@ -399,11 +397,13 @@ LOOPVQ_API loopvq_status loopvq_decode_attn_steps(const loopvq_codebook_desc* de
  * Returns LOOPVQ_ERR_WORKSPACE_TOO_SMALL when the layout would need more than
  * the 8 MiB array (loopvq_decode_workspace_bytes tells how much it needs).
  * The first call on a device looks up the array's device address (a
- * cudaGetSymbolAddress with that device current); make that first call
- * before any stream capture.  Every call shares the one array per device:
- * each call zeroes its counters on `stream` before the kernel runs, and two
- * calls whose kernels overlap on the GPU (different streams, no ordering)
- * race on it and give wrong results.
+ * cudaGetSymbolAddress with that device current) and caches it for the life
+ * of the process; make that first call before any stream capture, and do not
+ * reset the device (cudaDeviceReset) between calls.  Every call shares the
+ * one array per device: every split writes its partial before the merge
+ * reads it, so nothing needs clearing, but two calls whose kernels overlap
+ * on the GPU (different streams, no ordering) race on it and give wrong
+ * results.
  */
 LOOPVQ_API loopvq_status loopvq_decode_attn_noalloc(const loopvq_codebook_desc* desc, const void* cbK_packed,
                                                     const void* cbV_packed, const loopvq_cache_layout* layout,

@@ -29,7 +29,7 @@ class DecodeCache:
     def __init__(self, *, n_loop, tc, n_heads_kv, head_dim, group_elems, ctx_lens, n_sink=64, n_recent=256,
                  page=8, n_codes=256, n_heads_q=None, cb_dtype=torch.bfloat16, q_dtype=torch.bfloat16,
                  out_dtype=torch.float32, device="cuda", max_ctx_len=None, pool_slack_tokens=0,
-                 static_inputs=False, static_windows=False):
+                 static_inputs=False):
         self.device = torch.device(device)
         self.T, self.Tc, self.H, self.D, self.G = n_loop, tc, n_heads_kv, head_dim, group_elems
         self.Hq = n_heads_q or n_heads_kv
@@ -71,12 +71,9 @@ class DecodeCache:
         self.ctx_dev = torch.tensor(self.ctx_lens, dtype=torch.int32, device=dev)
         self.body_off_dev = torch.tensor(body_off, dtype=torch.int64, device=dev)
         self.win_off_dev = torch.tensor(win_off, dtype=torch.int64, device=dev)
-        # static_inputs: this cache's layout arrays, pools and codebooks are not
-        # written by kernels that may still run when a decode starts;
-        # static_windows: nor its window pools (the current token then comes
-        # through decode(new_k=..., new_v=...))
-        self.flags = ((L.LOOPVQ_LAYOUT_STATIC_INPUTS if static_inputs else 0) |
-                      (L.LOOPVQ_LAYOUT_STATIC_WINDOWS if static_inputs and static_windows else 0))
+        # static_inputs: this cache's layout arrays, index pools and codebooks
+        # are not written by kernels that may still run when a decode starts
+        self.flags = L.LOOPVQ_LAYOUT_STATIC_INPUTS if static_inputs else 0
         self.layout = self._make_layout(None, None)
         ws = L.loopvq_decode_workspace_bytes(self.desc, self.layout)
         if ws == 0:

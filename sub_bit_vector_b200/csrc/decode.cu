@@ -93,7 +93,6 @@ struct DecodeParams {
   int out_bf16;
   float* lse;
   uint32_t* status;
-  uint32_t* tickets;
   float* partials;
   // Several loop steps in one launch: step loop_step + i for i < n_steps;
   // queries, outputs, lse and partials are [n_steps][batch][Hq]..., the
@@ -104,7 +103,6 @@ struct DecodeParams {
   int split_len;   // body tokens per split (multiple of 32, <= the kernel's cap)
   int max_splits;  // grid.x
   int static_inputs;  // layout arrays, index pools and codebooks are not being written by earlier kernels
-  int static_windows;  // nor the window pools
   // paged body: body token p at pool position body_pages[r][p / bpt] * bpt + p % bpt
   int paged;
   const int32_t* body_pages;
@@ -436,7 +434,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
     const int64_t idx_blk = (int64_t)((p.loop_step + sidx) / p.Tc - p.loop_step / p.Tc) * p.idx_blk_bytes;
     const uint32_t vslice_bytes = (uint32_t)(p.C * D * sizeof(CBT));
     if (leader && !is_window && n_tok > 0) prefetch_l2(vslice, vslice_bytes);  // the epilogue's codebook slice
-    if (is_window && p.static_inputs && !p.static_windows) griddep_wait();  // rows may come from that kernel
+    // window rows may be written by the kernels before this one (an earlier
+    // decode call of the same cache stores its new token there)
+    if (is_window && p.static_inputs) griddep_wait();
     const int n_slice = (is_window || n_tok == 0) ? 0 : (int)((vslice_bytes + kStageBytes - 1) / kStageBytes);
     const int32_t* pages = p.paged ? p.body_pages + (size_t)r * p.max_body_pages : nullptr;
     const int64_t n_phys = p.paged ? p.body_pool_tokens / p.body_page_tokens : 0;
@@ -957,7 +957,8 @@ static int max_body_tokens(const loopvq_cache_layout* L) {
 // workspace bound independent of the device: plan with a generous SM count
 static WsLayout decode_ws(const Geo& g, const loopvq_cache_layout* L, int n_steps = 1) {
   const int64_t units = (int64_t)L->batch * g.Hq * n_steps;
-  DecodePlan pl = decode_plan(units, max_body_tokens(L), 1024);
+  const int cap = long_splits(g.D, (int)cb_elem_bytes(g)) ? kSplitCapLong : kSplitCap;
+  DecodePlan pl = decode_plan(units, max_body_tokens(L), 1024, cap);
   return ws_layout(units, pl.max_splits, g.D);
 }
 
@@ -965,8 +966,7 @@ static loopvq_status check_layout(const loopvq_cache_layout* L) {
   if (!L || L->batch < 1 || L->n_sink < 0 || L->n_recent < 0 || L->page < 1 || L->max_ctx_len < 0)
     return LOOPVQ_ERR_INVALID_ARG;
   const bool paged = L->flags & LOOPVQ_LAYOUT_PAGED_BODY, ring = L->flags & LOOPVQ_LAYOUT_RING_WINDOW;
-  if (L->flags & ~(LOOPVQ_LAYOUT_STATIC_INPUTS | LOOPVQ_LAYOUT_PAGED_BODY | LOOPVQ_LAYOUT_RING_WINDOW |
-                   LOOPVQ_LAYOUT_STATIC_WINDOWS))
+  if (L->flags & ~(LOOPVQ_LAYOUT_STATIC_INPUTS | LOOPVQ_LAYOUT_PAGED_BODY | LOOPVQ_LAYOUT_RING_WINDOW))
     return LOOPVQ_ERR_INVALID_ARG;
   if (!L->ctx_len || !L->win_off || (!paged && !L->body_off)) return LOOPVQ_ERR_INVALID_ARG;
   if (L->body_pool_tokens < 0 || (L->body_pool_tokens & 31) || L->win_pool_tokens < 0) return LOOPVQ_ERR_INVALID_ARG;
@@ -986,7 +986,6 @@ static loopvq_status check_layout(const loopvq_cache_layout* L) {
 
 // Layout fields of the kernel parameters shared by both entry points.
 static void fill_layout_params(DecodeParams& p, const loopvq_cache_layout* L) {
-  p.static_windows = ((L->flags & LOOPVQ_LAYOUT_STATIC_WINDOWS) && (L->flags & LOOPVQ_LAYOUT_STATIC_INPUTS)) ? 1 : 0;
   p.paged = (L->flags & LOOPVQ_LAYOUT_PAGED_BODY) ? 1 : 0;
   p.body_pages = L->body_pages;
   p.body_page_tokens = p.paged ? L->body_page_tokens : 32;
@@ -1114,7 +1113,6 @@ static loopvq_status decode_with_workspace(const loopvq_codebook_desc* desc, con
   const WsLayout ws = decode_ws(g, layout, n_steps);
   if (workspace_bytes < ws.total) return LOOPVQ_ERR_WORKSPACE_TOO_SMALL;
   p.status = (uint32_t*)workspace;
-  p.tickets = (uint32_t*)((uint8_t*)workspace + ws.tickets_off);
   p.partials = (float*)((uint8_t*)workspace + ws.partials_off);
   return decode_launch(g, p, (cudaStream_t)stream);
 }
@@ -1222,11 +1220,10 @@ extern "C" loopvq_status loopvq_decode_attn_noalloc(const loopvq_codebook_desc* 
 
   void* scratch = nullptr;
   if ((st = static_scratch(&scratch)) != LOOPVQ_OK) return st;
-  cudaStream_t s = (cudaStream_t)stream;
-  // the status word and the split counters must start at zero
-  if (cudaMemsetAsync(scratch, 0, ws.partials_off, s) != cudaSuccess) return LOOPVQ_ERR_CUDA;
-  p.status = fault_bits ? fault_bits : (uint32_t*)scratch;
-  p.tickets = (uint32_t*)((uint8_t*)scratch + ws.tickets_off);
+  // every split writes its partial before the merge kernel reads it, so
+  // nothing in the array needs clearing; faults go to the caller's word (or
+  // nowhere when fault_bits is null)
+  p.status = fault_bits;
   p.partials = (float*)((uint8_t*)scratch + ws.partials_off);
-  return decode_launch(g, p, s);
+  return decode_launch(g, p, (cudaStream_t)stream);
 }

@@ -183,7 +183,8 @@ __global__ void __launch_bounds__(kSmallWarps * 32) encode_small_kernel(const En
 }
 
 bool encode_tc_try(const Geo& g, const void* cb, int kind, const void* x, int64_t n_tokens, int64_t st, int64_t sn,
-                   int64_t sh, uint8_t* pool, int64_t tok_off, int64_t pool_tokens, cudaStream_t s, cudaError_t* err);
+                   int64_t sh, uint8_t* pool, int64_t tok_off, int64_t pool_tokens, uint32_t* faults, cudaStream_t s,
+                   cudaError_t* err);
 
 // Below this many tokens a 128-row tensor-core tile or a 256-thread chunk is
 // mostly padding, and the few-token kernel runs instead.
@@ -196,7 +197,7 @@ using namespace loopvq;
 extern "C" loopvq_status loopvq_encode(const loopvq_codebook_desc* desc, const void* cb_packed, loopvq_kind kind,
                                        const void* x, loopvq_dtype x_dtype, int64_t n_tokens, int64_t stride_t,
                                        int64_t stride_n, int64_t stride_h, uint8_t* idx_pool, int64_t tok_off,
-                                       int64_t pool_tokens, loopvq_stream_t stream) {
+                                       int64_t pool_tokens, uint32_t* fault_bits, loopvq_stream_t stream) {
   Geo g;
   loopvq_status st = make_geo(desc, &g);
   if (st != LOOPVQ_OK) return st;
@@ -206,7 +207,8 @@ extern "C" loopvq_status loopvq_encode(const loopvq_codebook_desc* desc, const v
     return LOOPVQ_ERR_INVALID_ARG;
   if (stride_t < 0 || stride_n < 0 || stride_h < 0) return LOOPVQ_ERR_INVALID_ARG;
   if (n_tokens == 0) return LOOPVQ_OK;
-  if (!cb_packed || !x || !idx_pool || ((uintptr_t)cb_packed & 15)) return LOOPVQ_ERR_INVALID_ARG;
+  if (!cb_packed || !x || !idx_pool || ((uintptr_t)cb_packed & 15) || ((uintptr_t)fault_bits & 3))
+    return LOOPVQ_ERR_INVALID_ARG;
 
   EncodeParams p;
   p.x = x; p.x_bf16 = x_dtype == LOOPVQ_BF16;
@@ -244,7 +246,7 @@ extern "C" loopvq_status loopvq_encode(const loopvq_codebook_desc* desc, const v
   if (p.x_bf16) {
     cudaError_t e = cudaSuccess;
     if (encode_tc_try(g, cb_packed, (int)kind, x, n_tokens, stride_t, stride_n, stride_h, idx_pool, tok_off,
-                      pool_tokens, s, &e))
+                      pool_tokens, fault_bits, s, &e))
       return e == cudaSuccess ? LOOPVQ_OK : LOOPVQ_ERR_CUDA;
   }
 #define LOOPVQ_ENC(GG, TT)                                                                       \

@@ -50,9 +50,8 @@ struct EncodeTcParams {
   int Tc, H, J, W, kind;
   uint8_t* pool;
   int64_t tok_off, pool_tokens;
+  uint32_t* faults;  // caller's fault word, or null
 };
-
-__device__ uint32_t g_encode_faults;
 
 // ---- canonical K-major, no-swizzle operand layout ---------------------------
 // A [rows][KP] bf16 operand is stored as 8-row x 16-byte core matrices of 128
@@ -257,7 +256,7 @@ __global__ void __launch_bounds__(kTcThreads, 2) encode_tc_kernel(const EncodeTc
     if (__syncthreads_or(!done)) {
       // never expected: record it, give the MMA one more bounded wait so no
       // tensor-core write is in flight, then leave (codes of this tile unwritten)
-      if (tid == 0) atomicOr(&g_encode_faults, LOOPVQ_FAULT_TIMEOUT);
+      if (tid == 0) set_fault(p.faults, LOOPVQ_FAULT_TIMEOUT);
       mbar_wait_bounded(smem_u32(mbar), phase);
       break;
     }
@@ -371,7 +370,8 @@ static cudaError_t launch_encode_tc(const EncodeTcParams& p, dim3 grid, cudaStre
 // codebooks with G in {16, 32} and W a multiple of 4.  Returns false (and
 // launches nothing) when the shape is not served.
 bool encode_tc_try(const Geo& g, const void* cb, int kind, const void* x, int64_t n_tokens, int64_t st, int64_t sn,
-                   int64_t sh, uint8_t* pool, int64_t tok_off, int64_t pool_tokens, cudaStream_t s, cudaError_t* err) {
+                   int64_t sh, uint8_t* pool, int64_t tok_off, int64_t pool_tokens, uint32_t* faults, cudaStream_t s,
+                   cudaError_t* err) {
   if (!g.cb_bf16 || g.C != kTcCodes || (g.G != 16 && g.G != 32) || (g.W & 3)) return false;
   if (((uintptr_t)x & 7) || (st & 3) || (sn & 3) || (sh & 3)) return false;
   const int64_t tiles = (n_tokens + kTcTile - 1) / kTcTile;
@@ -384,6 +384,7 @@ bool encode_tc_try(const Geo& g, const void* cb, int kind, const void* x, int64_
   p.cb = (const __nv_bfloat16*)cb;
   p.Tc = g.Tc; p.H = g.H; p.J = g.J; p.W = g.W; p.kind = kind;
   p.pool = pool; p.tok_off = tok_off; p.pool_tokens = pool_tokens;
+  p.faults = faults;
   // slot j fastest: the J CTAs of one token chunk run together and share its
   // sectors in L2
   dim3 grid(g.J, (unsigned)ctas_y, g.NB * g.H);
@@ -392,21 +393,3 @@ bool encode_tc_try(const Geo& g, const void* cb, int kind, const void* x, int64_
 }
 
 }  // namespace loopvq
-
-using namespace loopvq;
-
-extern "C" loopvq_status loopvq_read_encode_faults(uint32_t* bits, int32_t clear, loopvq_stream_t stream) {
-  uint32_t v = 0;
-  cudaStream_t s = (cudaStream_t)stream;
-  if (cudaMemcpyFromSymbolAsync(&v, g_encode_faults, sizeof(v), 0, cudaMemcpyDeviceToHost, s) != cudaSuccess)
-    return LOOPVQ_ERR_CUDA;
-  if (cudaStreamSynchronize(s) != cudaSuccess) return LOOPVQ_ERR_CUDA;
-  if (clear) {
-    const uint32_t z = 0;
-    if (cudaMemcpyToSymbolAsync(g_encode_faults, &z, sizeof(z), 0, cudaMemcpyHostToDevice, s) != cudaSuccess ||
-        cudaStreamSynchronize(s) != cudaSuccess)
-      return LOOPVQ_ERR_CUDA;
-  }
-  if (bits) *bits = v;
-  return v ? LOOPVQ_ERR_DEVICE_FAULT : LOOPVQ_OK;
-}

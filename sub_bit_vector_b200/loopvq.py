@@ -35,13 +35,12 @@ LOOPVQ_FAULT_TIMEOUT = 0x8
 LOOPVQ_LAYOUT_STATIC_INPUTS = 0x1
 LOOPVQ_LAYOUT_PAGED_BODY = 0x2
 LOOPVQ_LAYOUT_RING_WINDOW = 0x4
-LOOPVQ_LAYOUT_STATIC_WINDOWS = 0x8
 
 EXPORTED = [
     "loopvq_version", "loopvq_status_string", "loopvq_validate_desc", "loopvq_ctx_split",
     "loopvq_bits_per_element",
     "loopvq_codebook_packed_bytes", "loopvq_codebook_pack", "loopvq_index_pool_bytes",
-    "loopvq_index_pool_pack", "loopvq_index_pool_unpack", "loopvq_encode", "loopvq_read_encode_faults",
+    "loopvq_index_pool_pack", "loopvq_index_pool_unpack", "loopvq_encode",
     "loopvq_codebook_update_workspace_bytes", "loopvq_codebook_update", "loopvq_codebook_grad",
     "loopvq_decode_workspace_bytes", "loopvq_decode_attn", "loopvq_decode_attn_noalloc",
     "loopvq_decode_steps_workspace_bytes", "loopvq_decode_attn_steps",
@@ -100,8 +99,8 @@ def _load() -> ctypes.CDLL:
         "loopvq_index_pool_bytes": (SZ, [D, I64]),
         "loopvq_index_pool_pack": (ctypes.c_int, [D, ctypes.c_int, U8P, I64, U8P, I64, I64, P]),
         "loopvq_index_pool_unpack": (ctypes.c_int, [D, ctypes.c_int, U8P, I64, I64, I64, U8P, P]),
-        "loopvq_encode": (ctypes.c_int, [D, P, ctypes.c_int, P, ctypes.c_int, I64, I64, I64, I64, U8P, I64, I64, P]),
-        "loopvq_read_encode_faults": (ctypes.c_int, [ctypes.POINTER(ctypes.c_uint32), I32, P]),
+        "loopvq_encode": (ctypes.c_int, [D, P, ctypes.c_int, P, ctypes.c_int, I64, I64, I64, I64, U8P, I64, I64, P,
+                                         P]),
         "loopvq_codebook_update_workspace_bytes": (SZ, [D]),
         "loopvq_codebook_update": (ctypes.c_int, [D, ctypes.c_int, P, ctypes.c_int, I64, I64, I64, I64, U8P, I64, I64,
                                                   P, P, P, P, SZ, P]),
@@ -248,20 +247,13 @@ def loopvq_index_pool_unpack(desc, kind, pool, tok_off, pool_tokens, n_tokens, c
 
 
 def loopvq_encode(desc, cb_packed, kind, x, n_tokens, stride_t, stride_n, stride_h, idx_pool, tok_off,
-                  pool_tokens, stream=None, x_dtype=None) -> None:
+                  pool_tokens, stream=None, x_dtype=None, fault_bits=None) -> None:
+    """fault_bits: an int32/uint32 device tensor of one element that receives
+    the kernel's LOOPVQ_FAULT_* bits (OR-ed in), or None."""
     xd = _dtype_code(x) if x_dtype is None else x_dtype
     _check("loopvq_encode", _lib.loopvq_encode(
         ctypes.byref(desc), _ptr(cb_packed), kind, _ptr(x), xd, n_tokens, stride_t, stride_n, stride_h,
-        _ptr(idx_pool), tok_off, pool_tokens, _stream(stream)))
-
-
-def loopvq_read_encode_faults(clear=False, stream=None):
-    """Returns (status, fault_bits) of the encoder's device fault word; waits for the stream."""
-    bits = ctypes.c_uint32(0)
-    st = _lib.loopvq_read_encode_faults(ctypes.byref(bits), 1 if clear else 0, _stream(stream))
-    if st not in (LOOPVQ_OK, LOOPVQ_ERR_DEVICE_FAULT):
-        raise LoopVQError("loopvq_read_encode_faults", st)
-    return st, bits.value
+        _ptr(idx_pool), tok_off, pool_tokens, _ptr(fault_bits), _stream(stream)))
 
 
 def loopvq_codebook_update_workspace_bytes(desc) -> int:
