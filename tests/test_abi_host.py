@@ -26,6 +26,14 @@ def test_every_declared_symbol_is_exported_and_bound():
         assert callable(getattr(L, n)), n
 
 
+def test_library_keeps_no_encode_fault_word():
+    """Encode faults go to a word the caller passes; the library exports no
+    reader of a global one (its only global state is the allocation-free
+    decode's scratch array)."""
+    assert not hasattr(L._lib, "loopvq_read_encode_faults")
+    assert "loopvq_read_encode_faults" not in open(HEADER).read()
+
+
 def test_version_and_status_strings():
     assert "sm_100a" in L.loopvq_version()
     for s in range(6):
@@ -115,12 +123,15 @@ def test_encode_and_pool_reject_bad_arguments():
     d = L.make_desc(4, 4, 16, 128, 16)
     D = ctypes.byref(d)
     enc = L._lib.loopvq_encode
-    assert enc(D, FAKE, 0, FAKE, 1, 8, 1, 1, 1, FAKE, 30, 32, None) == L.LOOPVQ_ERR_INVALID_ARG  # past pool end
-    assert enc(D, FAKE, 2, FAKE, 1, 8, 1, 1, 1, FAKE, 0, 32, None) == L.LOOPVQ_ERR_INVALID_ARG   # bad kind
-    assert enc(D, FAKE, 0, FAKE, 3, 8, 1, 1, 1, FAKE, 0, 32, None) == L.LOOPVQ_ERR_INVALID_ARG   # bad dtype
-    assert enc(D, FAKE, 0, FAKE, 1, 8, -1, 1, 1, FAKE, 0, 32, None) == L.LOOPVQ_ERR_INVALID_ARG  # stride
-    assert enc(D, FAKE + 4, 0, FAKE, 1, 8, 1, 1, 1, FAKE, 0, 32, None) == L.LOOPVQ_ERR_INVALID_ARG  # align
-    assert enc(D, FAKE, 0, FAKE, 1, 0, 1, 1, 1, FAKE, 0, 32, None) == L.LOOPVQ_OK                 # empty
+    assert enc(D, FAKE, 0, FAKE, 1, 8, 1, 1, 1, FAKE, 30, 32, None, None) == L.LOOPVQ_ERR_INVALID_ARG  # past pool end
+    assert enc(D, FAKE, 2, FAKE, 1, 8, 1, 1, 1, FAKE, 0, 32, None, None) == L.LOOPVQ_ERR_INVALID_ARG   # bad kind
+    assert enc(D, FAKE, 0, FAKE, 3, 8, 1, 1, 1, FAKE, 0, 32, None, None) == L.LOOPVQ_ERR_INVALID_ARG   # bad dtype
+    assert enc(D, FAKE, 0, FAKE, 1, 8, -1, 1, 1, FAKE, 0, 32, None, None) == L.LOOPVQ_ERR_INVALID_ARG  # stride
+    assert enc(D, FAKE + 4, 0, FAKE, 1, 8, 1, 1, 1, FAKE, 0, 32, None, None) == L.LOOPVQ_ERR_INVALID_ARG  # align
+    assert enc(D, FAKE, 0, FAKE, 1, 0, 1, 1, 1, FAKE, 0, 32, None, None) == L.LOOPVQ_OK           # empty
+    # the fault word is the caller's: a misaligned one is refused before any launch
+    assert enc(D, FAKE, 0, FAKE, 1, 8, 1, 1, 1, FAKE, 0, 32, FAKE + 2, None) == L.LOOPVQ_ERR_INVALID_ARG
+    assert enc(D, FAKE, 0, FAKE, 1, 0, 1, 1, 1, FAKE, 0, 32, FAKE, None) == L.LOOPVQ_OK
     pack = L._lib.loopvq_index_pool_pack
     assert pack(D, 0, FAKE, 10, FAKE, 30, 32, None) == L.LOOPVQ_ERR_INVALID_ARG
     assert pack(D, 0, FAKE, 10, FAKE, 0, 33, None) == L.LOOPVQ_ERR_INVALID_ARG
@@ -194,7 +205,7 @@ def test_decode_steps_rejects_bad_step_ranges():
     d = L.make_desc(4, 2, 16, 128, 8)
     lay = _layout()
     D, Lp = ctypes.byref(d), ctypes.byref(lay)
-    assert L._lib.loopvq_decode_steps_workspace_bytes(D, Lp, 4) > L._lib.loopvq_decode_steps_workspace_bytes(D, Lp, 1)
+    assert L._lib.loopvq_decode_steps_workspace_bytes(D, Lp, 4) >= L._lib.loopvq_decode_steps_workspace_bytes(D, Lp, 1)
     assert L._lib.loopvq_decode_steps_workspace_bytes(D, Lp, 1) == L._lib.loopvq_decode_workspace_bytes(D, Lp)
     assert L._lib.loopvq_decode_steps_workspace_bytes(D, Lp, 5) == 0
     assert L._lib.loopvq_decode_steps_workspace_bytes(D, Lp, 0) == 0

@@ -181,6 +181,46 @@ def test_split_boundaries_and_multi_split_merge():
         case.check(t)
 
 
+def test_more_than_32_splits_merge_online():
+    """Batch 1, one KV head (GQA 1), 32K context: the planner spreads the one
+    (request, head) over more than 32 splits, so the merge kernel combines
+    them online, 32 partials at a time."""
+    case = Case(seed=8, ctx_lens=[32768], H=1)
+    _, L = _lib()
+    ws = L.loopvq_decode_workspace_bytes(case.c.desc, case.c.layout)
+    partials_off = 512          # status word block + one 256-byte block of counters
+    max_splits = (ws - partials_off) // ((case.D + 4) * 4)
+    assert max_splits > 32, max_splits
+    for t in range(4):
+        case.check(t)
+
+
+def _scores_max_weight(case, t, r, hq):
+    """Largest softmax weight of (request r, query head hq) at step t, from the
+    oracle's dequantized cache (a property of the inputs, not a result)."""
+    wk, _, ck, _ = case.req[r]
+    h = hq // (case.Hq // case.H)
+    K = O.dequantize(ck, case.cbk, t, case.Tc)[:, h]
+    keys = np.concatenate([wk[t][h], K]) if wk[t].shape[1] else K
+    s = keys.astype(np.float64) @ case.q[t, r, hq].astype(np.float64) * case.D ** -0.5
+    return float(np.exp(s.max() - (s.max() + np.log(np.sum(np.exp(s - s.max()))))))
+
+
+@pytest.mark.parametrize("qscale", [8.0, 32.0])
+def test_peaked_softmax_fixed_point_histogram(qscale):
+    """Queries scaled by 8 and 32 against keys with heavy-tailed outlier
+    channels: a few tokens carry most of the softmax mass and nearly every
+    other weight is far below one unit of the u32 fixed point (2^-S of the
+    split maximum), so the dithered rounding carries the tail.  Element by
+    element against the oracle at 2e-3."""
+    case = Case(seed=9, ctx_lens=[9000, 33000], H=2)
+    case.q = (case.q * qscale).astype(np.float32)   # a power of two: still exact bf16 values
+    peaked = max(_scores_max_weight(case, 1, r, hq) for r in (0, 1) for hq in range(case.Hq))
+    assert peaked > 0.2, peaked
+    for t in range(4):
+        case.check(t)
+
+
 @pytest.mark.parametrize("G,D,cbt", [(32, 64, torch.float32), (16, 64, torch.bfloat16), (32, 128, torch.float32),
                                      (8, 64, torch.float32)])
 def test_other_slot_counts(G, D, cbt):

@@ -98,16 +98,22 @@ def test_prefill_encode_32k_sampled(kind, tc, G):
     _accept(X, cb, tc, g[:, :, toks], tokens=toks)
 
 
-def test_tc4_beats_tc1_reconstruction_on_gpu_codes_sampled():
-    """Reports MSE (Tc=4 vs Tc=1 at 0.5 bit) of the oracle's codes on a sample;
-    directional check of the project page's loop-redundancy figure."""
-    X = _prefill("K")[:, :2048, :2]
+def test_tc4_beats_tc1_reconstruction_with_gpu_codes():
+    """Project page, "Method" loop-redundancy figure: at 0.5 bit a code
+    spanning 4 loop steps reconstructs loop-correlated keys with lower error
+    than a code spanning 1 step.  The codes are the GPU's (tensor-core
+    encode of bf16 inputs, each accepted against the oracle), dequantized by
+    the oracle."""
+    L = _L()
+    X = synth.round_bf16(_prefill("K")[:, :2048, :2])
     m = {}
     for tc in (4, 1):
-        cb = synth.codebook_from_rows(X, tc, 16, 256, seed=44)
-        idx, _, _ = O.encode(X, cb, tc)
-        m[tc] = O.reconstruction_mse(X, idx, cb, tc)
-    assert m[4] < m[1]
+        cb = synth.round_bf16(synth.codebook_from_rows(X, tc, 16, 256, seed=44))
+        desc = L.make_desc(4, tc, 2, 128, 16, 256)
+        g, _ = _encode_gpu(desc, cb, X, L.LOOPVQ_KEYS, 2048)
+        _accept(X, cb, tc, g)
+        m[tc] = O.reconstruction_mse(X, g, cb, tc)
+    assert m[4] < m[1], m
 
 
 def test_page_encode_from_window_pool_layout():
@@ -190,7 +196,9 @@ def test_tensor_core_encode_ragged_all_tokens(tc, G):
     L.loopvq_codebook_pack(desc, torch.from_numpy(cb).cuda().to(torch.bfloat16), packed)
     x_dev = torch.from_numpy(np.ascontiguousarray(X, dtype=np.float32)).cuda().to(torch.bfloat16)
     pool = torch.full((L.loopvq_index_pool_bytes(desc, pool_tokens),), 3, dtype=torch.uint8, device="cuda")
-    L.loopvq_encode(desc, packed, L.LOOPVQ_KEYS, x_dev, N, N * H * D, H * D, D, pool, tok_off, pool_tokens)
+    faults = torch.zeros(1, dtype=torch.int32, device="cuda")
+    L.loopvq_encode(desc, packed, L.LOOPVQ_KEYS, x_dev, N, N * H * D, H * D, D, pool, tok_off, pool_tokens,
+                    fault_bits=faults)
     J = D * tc // G
     allc = torch.zeros((T // tc, H, pool_tokens, J), dtype=torch.uint8, device="cuda")
     L.loopvq_index_pool_unpack(desc, L.LOOPVQ_KEYS, pool, 0, pool_tokens, pool_tokens, allc)
@@ -198,8 +206,7 @@ def test_tensor_core_encode_ragged_all_tokens(tc, G):
     a = allc.cpu().numpy().astype(np.int64)
     assert np.all(a[:, :, :tok_off] == 3) and np.all(a[:, :, tok_off + N:] == 3)
     _accept(X, cb, tc, a[:, :, tok_off:tok_off + N])
-    st, bits = L.loopvq_read_encode_faults(clear=True)
-    assert st == L.LOOPVQ_OK and bits == 0
+    assert int(faults.item()) == 0
 
 
 def test_tensor_core_encode_exact_ties_go_to_lowest_index():

@@ -14,6 +14,7 @@ import numpy as np
 import pytest
 import torch
 
+import oracle as O
 from sub_bit_vector_b200 import synth
 
 pytestmark = pytest.mark.gpu
@@ -33,12 +34,15 @@ def test_noalloc_matches_workspace_entry_on_two_calls():
     c = cache.DecodeCache(n_loop=T, tc=Tc, n_heads_kv=H, head_dim=D, group_elems=G, ctx_lens=ctx, n_heads_q=Hq)
     W, J = G // Tc, D * Tc // G
     outl = synth.key_outlier_channels(31, H, D)
-    c.set_codebooks(synth.uniform_codebook(32, 1, H, J, 256, Tc, W, outlier_channels=outl),
-                    synth.uniform_codebook(33, 1, H, J, 256, Tc, W))
+    cbk = synth.uniform_codebook(32, 1, H, J, 256, Tc, W, outlier_channels=outl)
+    cbv = synth.uniform_codebook(33, 1, H, J, 256, Tc, W)
+    c.set_codebooks(cbk, cbv)
+    reqs = []
     for r, (s, b, rc) in enumerate(c.splits):
         wk, wv, ck, cv = synth.decode_request(34 + r, T, H, D, J, 1, s + rc, b, outlier_channels=outl)
         c.set_request_window(r, wk, wv)
         c.set_request_codes(r, ck, cv)
+        reqs.append((wk, wv, ck, cv))
     q = synth.queries(35, T, len(ctx), Hq, D)
     out2 = torch.zeros_like(c.out)
     lse2 = torch.zeros_like(c.lse)
@@ -56,7 +60,28 @@ def test_noalloc_matches_workspace_entry_on_two_calls():
                 assert _err(got[r, h], ref[r, h]) <= TOL, (t, r, h)
         np.testing.assert_allclose(lgot, lref, atol=TOL, rtol=TOL)
         assert int(fault.item()) == 0
+        # and on its own against the fp64 oracle, request 0 (all query heads)
+        wk, wv, ck, cv = reqs[0]
+        o_ref, _ = O.decode_attention(q[t, 0], t, Tc, ck, cv, cbk, cbv, wk[t], wv[t], D ** -0.5)
+        for h in range(Hq):
+            assert _err(got[0, h], o_ref[h]) <= TOL, (t, h)
     assert c.device_status()[1] == 0
+
+    # a fault only the device can see lands in the caller's word: a context
+    # longer than the layout's max_ctx_len is reported and that request gets
+    # a zero output, the others are unaffected
+    bad_ctx = torch.tensor([ctx[0], c.max_ctx_len + 100, ctx[2], ctx[3]], dtype=torch.int32, device="cuda")
+    lay = L.make_layout(len(ctx), c.n_sink, c.n_recent, c.page, c.max_ctx_len, bad_ctx, c.body_off_dev,
+                        c.win_off_dev, c.body_pool_tokens, c.win_pool_tokens, 0)
+    fault.zero_()
+    L.loopvq_decode_attn_noalloc(c.desc, c.cbK, c.cbV, lay, c.idxK, c.idxV, c.winK, c.winV, c.q, 2,
+                                 D ** -0.5, out2, lse2, fault)
+    torch.cuda.synchronize()
+    assert int(fault.item()) & L.LOOPVQ_FAULT_CTX_RANGE
+    got = out2.cpu().numpy()
+    assert np.all(got[1] == 0) and np.all(np.isneginf(lse2.cpu().numpy()[1]))
+    for h in range(Hq):
+        assert _err(got[0, h], ref[0, h]) <= TOL
 
 
 def test_noalloc_refuses_layout_beyond_its_scratch():
