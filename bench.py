@@ -255,8 +255,7 @@ def build_layers(device, n_layers):
         # decode's own new_k/new_v write), so a launch may start streaming
         # them while the previous launch finishes
         c = cache.DecodeCache(n_loop=T, tc=TC, n_heads_kv=H, head_dim=D, group_elems=G, ctx_lens=[CTX],
-                              n_sink=N_SINK, n_recent=N_RECENT, page=PAGE, device=device, static_inputs=True,
-                              static_windows=True)
+                              n_sink=N_SINK, n_recent=N_RECENT, page=PAGE, device=device, static_inputs=True)
         outl = synth.key_outlier_channels(100 + i, H, D)
         c.set_codebooks(synth.uniform_codebook(200 + i, T // TC, H, J, 256, TC, W, outlier_channels=outl),
                         synth.uniform_codebook(300 + i, T // TC, H, J, 256, TC, W))
@@ -624,7 +623,7 @@ def run_gpu(args):
         for t in range(T):
             lay = L.make_layout(1, N_SINK, N_RECENT, PAGE, c.max_ctx_len, c.ctx_dev, c.body_off_dev, c.win_off_dev,
                                 c.body_pool_tokens, c.win_pool_tokens,
-                                L.LOOPVQ_LAYOUT_STATIC_INPUTS | L.LOOPVQ_LAYOUT_STATIC_WINDOWS,
+                                L.LOOPVQ_LAYOUT_STATIC_INPUTS,
                                 new_k=k_dev[t], new_v=v_dev[t])
             per.append(L.prepare_decode_attn(c.desc, c.cbK, c.cbV, lay, c.idxK, c.idxV, c.winK, c.winV, q_dev[t], t,
                                              D ** -0.5, out_dev[t], lse_dev[t], c.workspace, stream))
@@ -685,6 +684,135 @@ def run_gpu(args):
     return 0
 
 
+# ------------------------------------------------------------ profile cases
+# Small, self-contained launches of each kernel for a profiler:
+# ``python bench.py --profile-case NAME`` runs one case on cuda:0 and prints
+# its device status; inputs are seeded and drawn on the device, and each case
+# holds well under 2 GB so that a profiler replaying one launch stays small.
+#   decode       32768-token context, batch 1, 16 KV heads x 128, 4 loop
+#                steps, Tc = 4, G = 16 (0.5 bit): one launch per loop step
+#   decode-q     the same at G = 32 (0.25 bit)
+#   decode-gqa   8 KV heads, 16 query heads (GQA ratio 2), 4 launches
+#   decode-steps the decode case as one launch of all 4 loop steps, 2 launches
+#   encode       loop-axis encode of [4][32768][16][128] bf16, Tc = 4, G = 16
+#                (tensor-core kernel), 2 launches; encode-f32: fp32 input
+#                (CUDA-core kernel)
+#   residual     residual 4-bit coding of [4][32768][16][128] keys and values,
+#                then one decode per loop step
+#   page         encode of one 8-token page out of a [4][16][320][128] window
+
+def _pc_decode(G=16, Hkv=16, Hq=None):
+    import torch
+    from sub_bit_vector_b200 import cache, synth
+    c = cache.DecodeCache(n_loop=T, tc=TC, n_heads_kv=Hkv, head_dim=D, group_elems=G, ctx_lens=[CTX], n_heads_q=Hq)
+    W = G // TC
+    J = D // W
+    cb = synth.uniform_codebook(1, 1, Hkv, J, 256, TC, W)
+    c.set_codebooks(cb, cb)
+    c.idxK.copy_(synth.device_codes(2, c.idxK.numel()))
+    c.idxV.copy_(synth.device_codes(3, c.idxV.numel()))
+    c.winK.normal_()
+    c.winV.normal_()
+    c.q.normal_()
+    for t in range(T):
+        c.decode(t)
+    torch.cuda.synchronize()
+    print("decode status", c.device_status(), "algorithmic bytes per launch", c.algorithmic_bytes())
+
+
+def _pc_decode_steps():
+    import torch
+    from sub_bit_vector_b200 import cache, loopvq as L, synth
+    c = cache.DecodeCache(n_loop=T, tc=TC, n_heads_kv=H, head_dim=D, group_elems=G, ctx_lens=[CTX])
+    cb = synth.uniform_codebook(1, 1, H, D * TC // G, 256, TC, G // TC)
+    c.set_codebooks(cb, cb)
+    c.idxK.copy_(synth.device_codes(2, c.idxK.numel()))
+    c.idxV.copy_(synth.device_codes(3, c.idxV.numel()))
+    c.winK.normal_()
+    c.winV.normal_()
+    q = synth.device_normal(4, (T, 1, H, D)).to(torch.bfloat16)
+    out = torch.zeros((T, 1, H, D), dtype=torch.float32, device="cuda")
+    lse = torch.zeros((T, 1, H), dtype=torch.float32, device="cuda")
+    ws = torch.zeros(L.loopvq_decode_steps_workspace_bytes(c.desc, c.layout, T), dtype=torch.uint8, device="cuda")
+    for _ in range(2):
+        L.loopvq_decode_attn_steps(c.desc, c.cbK, c.cbV, c.layout, c.idxK, c.idxV, c.winK, c.winV, q, 0, T,
+                                   D ** -0.5, out, lse, ws)
+    torch.cuda.synchronize()
+    print("decode-steps status", L.loopvq_read_device_status(ws))
+
+
+def _pc_encode(dtype_name):
+    import torch
+    from sub_bit_vector_b200 import loopvq as L, synth
+    x = synth.device_normal(1, (T, CTX, H, D)).to(getattr(torch, dtype_name))
+    desc = L.make_desc(T, TC, H, D, G)
+    W = G // TC
+    cb = synth.device_normal(2, (T // TC, H, D // W, 256, TC, W))
+    packed = torch.zeros(L.loopvq_codebook_packed_bytes(desc), dtype=torch.uint8, device="cuda")
+    L.loopvq_codebook_pack(desc, cb, packed)
+    pool = torch.zeros(L.loopvq_index_pool_bytes(desc, CTX), dtype=torch.uint8, device="cuda")
+    faults = torch.zeros(1, dtype=torch.int32, device="cuda")
+    for _ in range(2):
+        L.loopvq_encode(desc, packed, L.LOOPVQ_KEYS, x, CTX, CTX * H * D, H * D, D, pool, 0, CTX, fault_bits=faults)
+    torch.cuda.synchronize()
+    print("encode fault bits", int(faults.item()))
+
+
+def _pc_residual():
+    import torch
+    from sub_bit_vector_b200 import loopvq as L, synth
+    desc = L.make_residual_desc(T, H, D)
+    bufs = []
+    for kind in (L.LOOPVQ_KEYS, L.LOOPVQ_VALUES):
+        codes = torch.zeros(L.loopvq_residual_codes_bytes(desc, CTX), dtype=torch.uint8, device="cuda")
+        params = torch.zeros(L.loopvq_residual_params_bytes(desc, kind, CTX) // 2, dtype=torch.float16, device="cuda")
+        x = synth.device_normal(20 + kind, (T, CTX, H, D))
+        L.loopvq_residual_encode(desc, kind, x, CTX, CTX * H * D, H * D, D, codes, params, 0, CTX)
+        bufs.append((codes, params))
+        del x
+    ctx = torch.tensor([CTX], dtype=torch.int32, device="cuda")
+    off = torch.zeros(1, dtype=torch.int64, device="cuda")
+    q = synth.device_normal(30, (1, H, D))
+    out = torch.zeros((1, H, D), dtype=torch.float32, device="cuda")
+    ws = torch.zeros(L.loopvq_residual_decode_workspace_bytes(desc, 1, CTX), dtype=torch.uint8, device="cuda")
+    for t in range(T):
+        L.loopvq_residual_decode_attn(desc, 1, CTX, ctx, off, CTX, bufs[0][0], bufs[0][1], bufs[1][0], bufs[1][1],
+                                      q, t, D ** -0.5, out, None, ws)
+    torch.cuda.synchronize()
+    print("residual decode status", L.loopvq_read_device_status(ws))
+
+
+def _pc_page():
+    import torch
+    from sub_bit_vector_b200 import loopvq as L, synth
+    P = 320
+    win = synth.device_normal(3, (T, H, P, D))
+    desc = L.make_desc(T, TC, H, D, G)
+    W = G // TC
+    cb = synth.device_normal(2, (T // TC, H, D // W, 256, TC, W))
+    packed = torch.zeros(L.loopvq_codebook_packed_bytes(desc), dtype=torch.uint8, device="cuda")
+    L.loopvq_codebook_pack(desc, cb, packed)
+    pool = torch.zeros(L.loopvq_index_pool_bytes(desc, 32), dtype=torch.uint8, device="cuda")
+    faults = torch.zeros(1, dtype=torch.int32, device="cuda")
+    for _ in range(4):
+        L.loopvq_encode(desc, packed, L.LOOPVQ_KEYS, win[:, :, 64:72], 8, H * P * D, D, P * D, pool, 0, 32,
+                        fault_bits=faults)
+    torch.cuda.synchronize()
+    print("page encode fault bits", int(faults.item()))
+
+
+PROFILE_CASES = {
+    "decode": lambda: _pc_decode(16),
+    "decode-q": lambda: _pc_decode(32),
+    "decode-gqa": lambda: _pc_decode(16, Hkv=8, Hq=16),
+    "decode-steps": _pc_decode_steps,
+    "encode": lambda: _pc_encode("bfloat16"),
+    "encode-f32": lambda: _pc_encode("float32"),
+    "page": _pc_page,
+    "residual": _pc_residual,
+}
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -694,7 +822,12 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extras", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--profile-case", choices=sorted(PROFILE_CASES), default=None,
+                    help="run one small launch set of a kernel for a profiler and exit")
     args = ap.parse_args(argv)
+    if args.profile_case:
+        PROFILE_CASES[args.profile_case]()
+        return 0
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":

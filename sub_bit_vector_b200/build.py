@@ -1,10 +1,11 @@
 """Builds libloopvq.so in-tree with nvcc for sm_100a.
 
-    python -m sub_bit_vector_b200.build [--debug]
+    python -m sub_bit_vector_b200.build [--force] [--ptxas-v]
 
 Every ``csrc/*.cu`` is compiled with ``-gencode arch=compute_100a,code=sm_100a``
 and linked (static CUDA runtime) into ``sub_bit_vector_b200/libloopvq.so``.
-Rebuilds only when a source or header is newer than the library.
+Rebuilds only when a source or header is newer than the library (--force
+rebuilds anyway; --ptxas-v prints ptxas register and spill reports).
 """
 from __future__ import annotations
 
