@@ -107,21 +107,6 @@ def cpu_baseline(budget_s: float = 15.0):
                       f"single_core_value from the median warm-up task"}
 
 
-def encode_oracle_sample(x_host, cb_host):
-    """The oracle's nearest-codeword encode timed on a seeded 1/64 sample of
-    the prefill's tokens (all heads and slots), one process; sub-vectors/s."""
-    import numpy as np
-    import oracle as O
-    rng = np.random.Generator(np.random.PCG64(11))
-    toks = np.sort(rng.choice(x_host.shape[1], x_host.shape[1] // 64, replace=False))
-    xs = x_host[:, toks]
-    t0 = time.perf_counter()
-    O.encode(xs, cb_host, TC)
-    wall = time.perf_counter() - t0
-    n_sub = (T // TC) * H * (D // (G // TC)) * len(toks)
-    return n_sub / wall, f"{len(toks)} of {x_host.shape[1]} tokens (1/64, all heads and slots), 1 process"
-
-
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -456,38 +441,153 @@ def residual_measurement(device, n_layers=4, reps=40):
                     "from t+1 planes; batch 1, 16x128, ctx 32768"}
 
 
-def encode_measurement(device, with_oracle, reps=5):
-    """Loop-axis encode of a 32768-token prefill's keys [4][32768][16][128]
-    bf16 at 0.5 bit (tensor-core kernel); with_oracle adds the oracle's rate
-    on a 1/64 sample (host cores)."""
+def encode_measurement(device, with_oracle, sm_mhz=None, reps=5):
+    """Prefill encode on its stated inputs: loop-correlated (rho = 0.9) bf16
+    keys (4 heavy-tailed outlier channels per head) and values
+    [4][32768][16][128], codebooks of seeded data rows, encoded at 0.5 bit
+    (G = 16) and 0.25 bit (G = 32) with Tc = 4, and at 0.5 bit with Tc = 1 (16
+    channels of one step) for the reconstruction comparison.  Per tensor: ms,
+    the fraction of the argmin ALU floor (2 integer operations per candidate
+    codeword on 148 SMs x 128 lanes at the SM clock) and of the HBM floor
+    (bf16 input + codes at the measured copy bandwidth).  with_oracle adds,
+    on a seeded 1/64 token sample on the host: the reconstruction MSE of the
+    GPU's codes (dequantized by the oracle) and the oracle's encode rate."""
+    import numpy as np
     import torch
     from sub_bit_vector_b200 import loopvq as L, synth
-    W = G // TC
+    peak, _ = _peak_hbm()
+    f_hz = (sm_mhz or 1965.0) * 1e6
+    rng = np.random.Generator(np.random.PCG64(11))
+    toks = np.sort(rng.choice(CTX, CTX // 64, replace=False))
+    out = {"what": "[4][32768][16][128] bf16 K (4 outlier channels x8) and V, rho 0.9, data-row codebooks; "
+                   "MSE on a 1/64 token sample (GPU codes, oracle dequantization)",
+           "alu_floor": "2 ops per candidate codeword / (148 SMs x 128 lanes x SM clock); alu_pipe_floor: the "
+                        "same over the integer ALU pipe's 64 lanes per clock, which min/max and key formation use",
+           "tensors": []}
+    for kind_name, seed, n_out in (("K", 40, 4), ("V", 41, 0)):
+        X = synth.loop_correlated(seed=seed, n_loop=T, n_tokens=CTX, n_heads=H, head_dim=D, n_outlier=n_out)
+        x_dev = torch.from_numpy(X).to(device).to(torch.bfloat16)
+        kind = L.LOOPVQ_KEYS if kind_name == "K" else L.LOOPVQ_VALUES
+        mse = {}
+        for tc, g in ((4, 16), (4, 32), (1, 16)):
+            cb = synth.codebook_from_rows(X, tc, g, 256, seed=seed + 2 + tc + g)
+            desc = L.make_desc(T, tc, H, D, g)
+            packed = torch.zeros(L.loopvq_codebook_packed_bytes(desc), dtype=torch.uint8, device=device)
+            L.loopvq_codebook_pack(desc, torch.from_numpy(cb).to(device).to(torch.bfloat16), packed)
+            pool = torch.zeros(L.loopvq_index_pool_bytes(desc, CTX), dtype=torch.uint8, device=device)
+            faults = torch.zeros(1, dtype=torch.int32, device=device)
+            args = (desc, packed, kind, x_dev, CTX, CTX * H * D, H * D, D, pool, 0, CTX)
+            for _ in range(2):
+                L.loopvq_encode(*args, fault_bits=faults)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            torch.cuda.synchronize()
+            e0.record()
+            for _ in range(reps):
+                L.loopvq_encode(*args, fault_bits=faults)
+            e1.record()
+            torch.cuda.synchronize()
+            ms = e0.elapsed_time(e1) / reps
+            J = D * tc // g
+            cand = (T // tc) * H * J * CTX * 256
+            alu_ms = cand * 2 / (148 * 128 * f_hz) * 1e3
+            alu_pipe_ms = cand * 2 / (148 * 64 * f_hz) * 1e3   # the integer ALU pipe's 64 lanes per clock
+            by = T * CTX * H * D * 2 + (T // tc) * H * J * CTX
+            hbm_ms = by / (peak * 1e9) * 1e3
+            rec = {"tensor": kind_name, "tc": tc, "group_elems": g, "bits": 8.0 / g, "ms_per_tensor": ms,
+                   "candidates": cand, "alu_floor_ms": alu_ms, "alu_floor_frac": alu_ms / ms,
+                   "alu_pipe_floor_ms": alu_pipe_ms, "alu_pipe_floor_frac": alu_pipe_ms / ms,
+                   "hbm_floor_ms": hbm_ms, "hbm_floor_frac": hbm_ms / ms, "fault_bits": int(faults.item())}
+            if with_oracle:
+                import oracle as O
+                codes = torch.zeros((T // tc, H, CTX, J), dtype=torch.uint8, device=device)
+                L.loopvq_index_pool_unpack(desc, kind, pool, 0, CTX, CTX, codes)
+                idx = codes.cpu().numpy()[:, :, toks].astype(np.int64)
+                xs = synth.round_bf16(X[:, toks])
+                rec["mse_sample"] = O.reconstruction_mse(xs, idx, synth.round_bf16(cb), tc)
+                mse[(tc, g)] = rec["mse_sample"]
+                if tc == 4 and g == 16 and kind_name == "K":
+                    t0 = time.perf_counter()
+                    O.encode(xs, synth.round_bf16(cb), tc)
+                    wall = time.perf_counter() - t0
+                    rec["oracle_subvectors_per_s"] = len(toks) * H * J / wall
+                    rec["oracle_sample"] = f"{len(toks)} of {CTX} tokens (1/64, all heads and slots), 1 process"
+            out["tensors"].append(rec)
+            del pool
+        if with_oracle:
+            out[f"mse_{kind_name}_tc4_over_tc1_at_half_bit"] = mse[(4, 16)] / mse[(1, 16)]
+        del x_dev
+    return out
+
+
+def decode_config_measurement(device, name, ctx_lens, group_elems, n_layers, reps):
+    """One decode configuration timed the way the headline is: a CUDA graph
+    of the 4 loop-step launches per layer, rotating over n_layers layer
+    caches (larger than L2 together), device-drawn codes, windows and
+    queries.  Returns us per launch, algorithmic bytes, GB/s, the fraction of
+    the measured HBM copy bandwidth and KV tokens/s."""
+    import torch
+    from sub_bit_vector_b200 import cache, synth
+    peak, _ = _peak_hbm()
+    W = group_elems // TC
     J = D // W
-    x = synth.device_normal(2100, (T, CTX, H, D), device=device)
-    cb = synth.device_normal(2101, (T // TC, H, J, 256, TC, W), device=device)
-    desc = L.make_desc(T, TC, H, D, G)
-    packed = torch.zeros(L.loopvq_codebook_packed_bytes(desc), dtype=torch.uint8, device=device)
-    L.loopvq_codebook_pack(desc, cb, packed)
-    pool = torch.zeros(L.loopvq_index_pool_bytes(desc, CTX), dtype=torch.uint8, device=device)
-    args = (desc, packed, L.LOOPVQ_KEYS, x, CTX, CTX * H * D, H * D, D, pool, 0, CTX)
-    for _ in range(2):
-        L.loopvq_encode(*args)
+    caches = []
+    for i in range(n_layers):
+        c = cache.DecodeCache(n_loop=T, tc=TC, n_heads_kv=H, head_dim=D, group_elems=group_elems, ctx_lens=ctx_lens,
+                              n_sink=N_SINK, n_recent=N_RECENT, page=PAGE, device=device, static_inputs=True)
+        outl = synth.key_outlier_channels(3100 + i, H, D)
+        c.set_codebooks(synth.uniform_codebook(3200 + i, T // TC, H, J, 256, TC, W, outlier_channels=outl),
+                        synth.uniform_codebook(3300 + i, T // TC, H, J, 256, TC, W))
+        c.idxK.copy_(synth.device_codes(3400 + i, c.idxK.numel(), device))
+        c.idxV.copy_(synth.device_codes(3500 + i, c.idxV.numel(), device))
+        c.winK.copy_(synth.device_normal(3600 + i, tuple(c.winK.shape), device=device))
+        c.winV.copy_(synth.device_normal(3700 + i, tuple(c.winV.shape), device=device))
+        c.q.copy_(synth.device_normal(3800 + i, tuple(c.q.shape), dtype=c.q.dtype, device=device))
+        caches.append(c)
+    s = torch.cuda.Stream(device)
+    with torch.cuda.stream(s):
+        for c in caches:
+            c.decode(0, stream=s)
+    torch.cuda.synchronize()
+    graphs = []
+    for c in caches:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s):
+            for t in range(T):
+                c.decode(t, stream=s)
+        graphs.append(g)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(s):
+        for i in range(2 * n_layers):
+            graphs[i % n_layers].replay()
+        torch.cuda.synchronize()
+        e0.record(s)
+        for i in range(reps):
+            graphs[i % n_layers].replay()
+        e1.record(s)
     torch.cuda.synchronize()
-    e0.record()
-    for _ in range(reps):
-        L.loopvq_encode(*args)
-    e1.record()
-    torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1) / reps
-    n_sub = (T // TC) * H * J * CTX
-    res = {"kernel": "loopvq::encode_tc_kernel<16,32>", "ms_per_tensor": ms, "subvectors_per_s": n_sub / (ms * 1e-3),
-           "what": "keys [4][32768][16][128] bf16, Tc=4, G=16, 256 codes"}
-    if with_oracle:
-        rate, sample = encode_oracle_sample(x.float().cpu().numpy(), cb.float().cpu().numpy())
-        res["oracle_subvectors_per_s"] = rate
-        res["oracle_sample"] = sample
+    us = e0.elapsed_time(e1) * 1e3 / (reps * T)
+    by = caches[0].algorithmic_bytes()
+    faults = max(c.device_status()[1] for c in caches)
+    del graphs, caches
+    torch.cuda.empty_cache()
+    return {"config": name, "bits": 8.0 / group_elems, "batch": len(ctx_lens), "kv_tokens": int(sum(ctx_lens)),
+            "us_per_launch": us, "algorithmic_bytes_per_launch": by, "GB_per_s": by / us / 1e3,
+            "frac_of_measured_hbm": by / us / 1e3 / peak, "kv_tokens_per_s": sum(ctx_lens) / (us * 1e-6),
+            "launches_timed": reps * T, "layer_caches": n_layers, "device_fault_bits": faults}
+
+
+def other_configs_measurement(device):
+    """The quarter-bit context sweep (4K..64K, batch 1) and the batch-128
+    ragged serving step (2048 + U{4096..16384} tokens per request, 0.5 bit),
+    each with the headline's timing method."""
+    from sub_bit_vector_b200 import synth
+    res = []
+    for ctx in (4096, 8192, 16384, 32768, 65536):
+        res.append(decode_config_measurement(device, f"0.25 bit, ctx {ctx}", [ctx], 32,
+                                             n_layers=8 if ctx <= 32768 else 4, reps=200))
+    ragged = [int(x) for x in synth.ragged_context_lengths(128)]
+    res.append(decode_config_measurement(device, "0.5 bit, batch 128 ragged (2048 + U[4096, 16384])", ragged, 16,
+                                         n_layers=2, reps=20))
     return res
 
 
@@ -664,9 +764,11 @@ def run_gpu(args):
             residual = residual_measurement(device)
         except Exception as exc:   # a context figure: report, never lose the line for it
             residual = {"error": f"{type(exc).__name__}: {exc}"}
+    others = other_configs_measurement(device) if not args.no_extras else None
     dense = dense_comparator(device) if not args.no_extras else None
     sdpa = sdpa_comparator(device) if not args.no_extras else None
-    enc = (encode_measurement(device, with_oracle=(rank == 0 and world == 1 and not args.no_cpu_baseline))
+    enc = (encode_measurement(device, with_oracle=(rank == 0 and world == 1 and not args.no_cpu_baseline),
+                              sm_mhz=clocks.get("sm_mhz"))
            if not args.no_extras else None)
     launches = args.steps * T * 2 + 2 * n_enc_steps   # decode + merge kernel per loop step; K and V page encodes
     if rank == 0:
@@ -675,7 +777,7 @@ def run_gpu(args):
                 "scaling": "weak", "vs_baseline": None, "dtype": "u8 codes, f32 accumulate", "data": "synthetic",
                 "config": dict(_config(), parallelism=f"replicas x{world}" if world > 1 else "single GPU"),
                 "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches,
-                "clocks": clocks, "all_steps_one_launch": steps_fused, "kv_residual_4bit": residual, "dense_bf16_comparator": dense, "torch_sdpa_bf16": sdpa, "encode": enc,
+                "clocks": clocks, "other_configs": others, "all_steps_one_launch": steps_fused, "kv_residual_4bit": residual, "dense_bf16_comparator": dense, "torch_sdpa_bf16": sdpa, "encode": enc,
                 "device_fault_bits": max(status)}
         print(json.dumps(line), flush=True)
     del decode_graphs, encode_graphs
