@@ -1,10 +1,11 @@
 // Dense bf16 split-K decode attention (sm_100a): the comparator that the
 // LoopVQ pages measure against (bf16 keys and values read for every token).
 //
-// One CTA per (split, query head, request); each of 16 warps streams its
-// share of the split's tokens, 4 tokens per iteration with all 8 row loads in
-// flight, and keeps an fp32 online softmax (log2 units); the warps merge in
-// shared memory and the last split of a (request, head) merges the splits.
+// One CTA per (split, query head, request), two CTAs per SM; each of 16
+// warps streams its share of the split's tokens, 6 tokens per iteration with
+// all 12 row loads in flight (about 100 KB of loads in flight per SM), and
+// keeps an fp32 online softmax (log2 units); the warps merge in shared memory
+// and the last split of a (request, head) merges the splits.
 
 #include "common.cuh"
 
@@ -12,7 +13,7 @@ namespace loopvq {
 
 constexpr int kDW = 16;
 constexpr int kDThreads = kDW * 32;
-constexpr int kDUnroll = 4;
+constexpr int kDUnroll = 6;
 
 struct DenseParams {
   int H, Hq, D, max_ctx, split_len, max_splits;
@@ -32,7 +33,7 @@ struct DenseParams {
 };
 
 template <int CPL>  // channels per lane: D / 32
-__global__ void __launch_bounds__(kDThreads) dense_decode_kernel(const DenseParams p) {
+__global__ void __launch_bounds__(kDThreads, 2) dense_decode_kernel(const DenseParams p) {
   __shared__ float wpart[kDW][CPL * 32 + 2];
   __shared__ float csm[2 * kMaxCombineSplits + kDThreads];
   __shared__ int flag;
@@ -155,7 +156,7 @@ __global__ void __launch_bounds__(kDThreads) dense_decode_kernel(const DensePara
 }
 
 static void dense_plan(int64_t units, int max_ctx, int n_sm, int* split_len, int* max_splits) {
-  int s = (int)(n_sm / (units > 0 ? units : 1));
+  int s = (int)(2 * n_sm / (units > 0 ? units : 1));  // two CTAs per SM
   const int cap = (max_ctx + 255) / 256;
   if (s > cap) s = cap;
   if (s < 1) s = 1;
