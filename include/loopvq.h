@@ -154,7 +154,7 @@ typedef struct {
   int32_t win_ring;           /* >= n_recent + page - 1 */
   int32_t reserved;           /* 0 */
   /* The current token's key and value at this loop step, device bf16
-   * [batch][n_heads_kv][head_dim], 8-byte aligned, or NULL.  When set, the
+   * [batch][n_heads_kv][head_dim], 4-byte aligned, or NULL.  When set, the
    * decode uses them for the current token (the last window token) and also
    * stores them in its window slot -- the pages' "write in bf16" fused into
    * attention. */
