@@ -652,6 +652,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
     }
   } else {
     // ---- LUT of step t: LUT[c][g*J + j] = sum_w q_{j*W+w} * B^K_t[c][j][w]
+    // The histogram later accumulates on top of these words (u32 adds wrap),
+    // so the thread keeps the bits it wrote and subtracts them at the end.
+    uint32_t lutb[kPer];
     {
       const int j = ctid % J;
       float qj[W];                 // q[j*W .. j*W+W) of this thread's slot j, log2 units
@@ -664,6 +667,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
 #pragma unroll
         for (int w = 0; w < W; ++w) acc = fmaf(qj[w], wk[k][w], acc);
         if (c >= p.C) acc = __int_as_float(0x7fc00000);  // NaN marks a code >= n_codes
+        lutb[k] = __float_as_uint(acc);
 #pragma unroll
         for (int g = 0; g < kCols / J; ++g) lut[c * kCols + g * J + j] = acc;
       }
@@ -721,9 +725,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
     consumer_sync();
     float m = -INFINITY;
     for (int w = 0; w < kNW; ++w) m = fmaxf(m, red[w]);
-    // the table is done with: the region becomes the histogram
-    for (int e = ctid; e < 256 * kCols / 4; e += kNW * 32) reinterpret_cast<uint4*>(hist)[e] = make_uint4(0u, 0u, 0u, 0u);
-    consumer_sync();
+    // the table is done with: the region becomes the histogram (no zeroing:
+    // every bin starts at the table word this thread wrote there)
     // fixed-point scale: n_tok * 2^S < 2^32 with S = clz(n_tok)
     const int S = __clz(max(n_tok, 1));
     const float scaleS = exp2f((float)S);
@@ -795,6 +798,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
         uint32_t hs = 0;
 #pragma unroll
         for (int g = 0; g < kCols / J; ++g) hs += hist[c * kCols + g * J + j];
+        hs -= (uint32_t)(kCols / J) * lutb[k];
         hf[k] = c < p.C ? (float)hs : 0.f;
       }
       float acc[W];
@@ -814,7 +818,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
       // bins of codes >= n_codes must be empty
       if (p.C < 256) {
         bool any = false;
-        for (int e = p.C * kCols + ctid; e < 256 * kCols; e += kNW * 32) any |= hist[e] != 0u;
+        for (int e = p.C * kCols + ctid; e < 256 * kCols; e += kNW * 32) any |= hist[e] != 0x7fc00000u;
         if (any) set_fault(p.status, LOOPVQ_FAULT_CODE_RANGE);
       }
       // lanes l and l + J of a warp hold the same slot: fold them first
