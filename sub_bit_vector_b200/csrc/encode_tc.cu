@@ -51,6 +51,10 @@ struct EncodeTcParams {
   uint8_t* pool;
   int64_t tok_off, pool_tokens;
   uint32_t* faults;  // caller's fault word, or null
+  // 256, passed at run time: the key's bits * 256 + code then issues as an
+  // integer multiply-add (FMA pipe) instead of a shift and add on the integer
+  // ALU pipe, which the top-2 min/max keep busy (measured 1.56 vs 1.65 ms)
+  uint32_t key_mul;
 };
 
 // ---- canonical K-major, no-swizzle operand layout ---------------------------
@@ -88,6 +92,28 @@ __device__ __forceinline__ void umma_commit(uint32_t mbar) {
 __device__ __forceinline__ void tmem_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tmem_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+// Waits for the outstanding TMEM loads and ties r to the wait, so that no use
+// of the loaded registers can be scheduled before it.
+__device__ __forceinline__ void tmem_wait_ld_tied(uint32_t (&r)[32]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+                 "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]),
+                 "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]),
+                 "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]),
+                 "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
+               :
+               : "memory");
+}
+__device__ __forceinline__ void tie_regs(uint32_t (&r)[32]) {
+  asm volatile(""
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+                 "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]),
+                 "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]),
+                 "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]),
+                 "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
+               :
+               : "memory");
+}
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
@@ -230,6 +256,15 @@ __global__ void __launch_bounds__(kTcThreads, 2) encode_tc_kernel(const EncodeTc
     // each within a few units of 2^-24 of the sum of the terms' magnitudes
     // (at most 2 (||x||^2 + ||c||^2)); taken as 2^-15 (||x||^2 + max ||c||^2).
     const float err = 3.0517578e-5f * (xx + nc_max);
+    // Keys quantize the fast distance at a power-of-two scale sk with
+    // d * sk < 2^22 (d <= (|x| + |c|)^2 + 2 err <= 2 (||x||^2 + max ||c||^2) + 2 err):
+    // fma(d, sk, 2^23) holds round(d * sk) in its low 23 bits, and
+    // bits * 256 + column puts the column below it -- one FFMA and one
+    // integer multiply-add per candidate, off the integer ALU pipe.
+    int ek = (int)((__float_as_uint(2.f * (xx + nc_max) + 4.f * err) >> 23) & 0xFFu) - 127;
+    ek = max(ek, -100);
+    const float sk = __uint_as_float((uint32_t)(21 - ek + 127) << 23);
+    const float inv_sk = __uint_as_float((uint32_t)(ek - 21 + 127) << 23);
     {
       // the row's norm carries a bias of 2 err, equal for every codeword, so
       // the fast distances stay positive and order as signed integers
@@ -263,47 +298,77 @@ __global__ void __launch_bounds__(kTcThreads, 2) encode_tc_kernel(const EncodeTc
     phase ^= 1u;
     tmem_fence_after();
 
-    // top-2 keys: within a 32-column chunk the key carries the column in its
-    // low 5 bits (an immediate); the chunk number joins in bits 5..7 when a
-    // chunk's top-2 merges into the row's
-    int k1 = 0x7FFFFFFF, k2 = 0x7FFFFFFF;
-#pragma unroll 1
-    for (int cc = 0; cc < kTcCodes / 32; cc += 2) {
-      uint32_t r[2][32];
-      tmem_ld32(t_row + (uint32_t)(cc * 32), r[0]);
-      tmem_ld32(t_row + (uint32_t)(cc * 32 + 32), r[1]);
-      tmem_wait_ld();
+    // top-2 keys over the 256 codes, 64 TMEM columns at a time (the next 64
+    // load while these are scanned); 8 independent chains of candidate pairs,
+    // a pair (lo <= hi) merging into a chain's sorted (x1 <= x2) as
+    // x2 = min(max(x1, lo), x2, hi), x1 = min(x1, lo); the code is the key's
+    // low byte (an immediate)
+    auto qkey = [&](uint32_t v, uint32_t code) -> int {
+      const float y = __fmaf_rn(__uint_as_float(v), sk, 8388608.f);
+      return (int)(__float_as_uint(y) * p.key_mul + code);
+    };
+    int x1[4], x2[4];
 #pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        // two chains of candidate pairs; a pair (lo <= hi) merges into a
-        // chain's sorted (x1 <= x2) as x2 = min(max(x1, lo), x2, hi), x1 = min(x1, lo)
-        int a1 = 0x7FFFFFFF, a2 = 0x7FFFFFFF, b1 = 0x7FFFFFFF, b2 = 0x7FFFFFFF;
+    for (int c = 0; c < 4; ++c) { x1[c] = 0x7FFFFFFF; x2[c] = 0x7FFFFFFF; }
+    uint32_t rb[2][2][32];
+    tmem_ld32(t_row, rb[0][0]);
+    tmem_ld32(t_row + 32u, rb[0][1]);
+    tmem_wait_ld_tied(rb[0][0]);
+    tie_regs(rb[0][1]);
 #pragma unroll
-        for (int q = 0; q < 32; q += 4) {
-          const int ka0 = (int)((r[u][q] & 0xFFFFFF00u) | (uint32_t)q);
-          const int ka1 = (int)((r[u][q + 1] & 0xFFFFFF00u) | (uint32_t)(q + 1));
-          const int kb0 = (int)((r[u][q + 2] & 0xFFFFFF00u) | (uint32_t)(q + 2));
-          const int kb1 = (int)((r[u][q + 3] & 0xFFFFFF00u) | (uint32_t)(q + 3));
-          const int alo = min(ka0, ka1), ahi = max(ka0, ka1);
-          const int blo = min(kb0, kb1), bhi = max(kb0, kb1);
-          a2 = __vimin3_s32(max(a1, alo), a2, ahi);
-          a1 = min(a1, alo);
-          b2 = __vimin3_s32(max(b1, blo), b2, bhi);
-          b1 = min(b1, blo);
-        }
-        const int chunk = (cc + u) << 5;
-        const int c1 = min(a1, b1) | chunk, c2 = min(max(a1, b1), min(a2, b2)) | chunk;
-        k2 = min(max(k1, c1), min(k2, c2));
-        k1 = min(k1, c1);
+    for (int i = 0; i < kTcCodes / 64; ++i) {
+      uint32_t (&cur)[2][32] = rb[i & 1];
+      uint32_t (&nxt)[2][32] = rb[(i + 1) & 1];
+      if (i + 1 < kTcCodes / 64) {
+        tmem_ld32(t_row + (uint32_t)(64 * i + 64), nxt[0]);
+        tmem_ld32(t_row + (uint32_t)(64 * i + 96), nxt[1]);
+      }
+#pragma unroll
+      for (int pp = 0; pp < 32; ++pp) {
+        const int col = 2 * pp;
+        const int k0 = qkey(cur[col >> 5][col & 31], (uint32_t)(64 * i + col));
+        const int k1v = qkey(cur[(col + 1) >> 5][(col + 1) & 31], (uint32_t)(64 * i + col + 1));
+        const int lo = min(k0, k1v), hi = max(k0, k1v);
+        const int c = pp & 3;
+        x2[c] = min(min(max(x1[c], lo), x2[c]), hi);
+        x1[c] = min(x1[c], lo);
+      }
+      if (i + 1 < kTcCodes / 64) {
+        tmem_wait_ld_tied(nxt[0]);
+        tie_regs(nxt[1]);
       }
     }
+    // the row's two smallest keys: k1 is the smallest chain head; k2 the
+    // smallest of the other heads and of every chain's second
+    const int k1 = min(min(x1[0], x1[1]), min(x1[2], x1[3]));
+    int k2 = min(min(x2[0], x2[1]), min(x2[2], x2[3]));
+#pragma unroll
+    for (int c = 0; c < 4; ++c) k2 = min(k2, x1[c] != k1 ? x1[c] : 0x7FFFFFFF);
     int code = k1 & 0xFF;
-    const float d1 = __int_as_float(k1 & (int)0xFFFFFF00u);
-    const float d2 = __int_as_float(k2 & (int)0xFFFFFF00u);
-    const bool refine = ok && !(d2 - d1 > 2.f * err + 6.1035156e-5f * d2);
+    // the gap of the two smallest keys in units of 1/sk; each key rounds by
+    // at most half a unit
+    const float gap = (float)((k2 >> 8) - (k1 >> 8));
+    const bool refine = ok && !(gap > 2.f * err * sk + 2.f);
     if (__any_sync(0xffffffffu, refine)) {
-      // every codeword whose fast distance is within 2 err of the minimum
-      const float thr = d1 * (1.f + 6.1035156e-5f) + 2.f * err;
+      // Only the codes whose fast distance is within 2 err of the minimum can
+      // be the nearest.  The third smallest chain value is the row's third
+      // smallest key unless the two smallest share a chain (then k2 is that
+      // chain's second); when it is farther than the bound from k1, the two
+      // codes of k1 and k2 are the only candidates and are solved directly,
+      // otherwise the row is scanned in full.
+      bool full = false;
+      if (refine) {
+        bool same = false;
+        int k3 = 0x7FFFFFFF;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          same |= x2[c] == k2;
+          k3 = min(k3, x1[c] > k2 ? x1[c] : 0x7FFFFFFF);
+          k3 = min(k3, x2[c] > k2 ? x2[c] : 0x7FFFFFFF);
+        }
+        full = same || !((float)((k3 >> 8) - (k1 >> 8)) > 2.f * err * sk + 2.f);
+      }
+      const float thr = (float)(k1 >> 8) * inv_sk + 2.f * err + 2.f * inv_sk;
       float xe[G];
 #pragma unroll
       for (int k8 = 0; k8 < G / 8; ++k8) {
@@ -312,38 +377,51 @@ __global__ void __launch_bounds__(kTcThreads, 2) encode_tc_kernel(const EncodeTc
 #pragma unroll
         for (int i = 0; i < 4; ++i) { xe[k8 * 8 + 2 * i] = bf16_lo(w[i]); xe[k8 * 8 + 2 * i + 1] = bf16_hi(w[i]); }
       }
-      float best = INFINITY;
-      int bi = code;
-#pragma unroll 1
-      for (int cc = 0; cc < kTcCodes / 32; ++cc) {
-        uint32_t r[32];
-        tmem_ld32(t_row + (uint32_t)(cc * 32), r);
-        tmem_wait_ld();
-        uint32_t cand = 0;
+      // exact fp32 distance sum_g (x_g - c_g)^2 to codeword c
+      auto exact_d = [&](int c) -> float {
+        float d = 0.f;
 #pragma unroll
-        for (int q = 0; q < 32; ++q) cand |= (__uint_as_float(r[q]) <= thr ? 1u : 0u) << q;
-        if (!refine) cand = 0;
-        while (cand) {
-          const int c = cc * 32 + __ffs(cand) - 1;
-          cand &= cand - 1;
-          float d = 0.f;
+        for (int k8 = 0; k8 < G / 8; ++k8) {
+          const uint4 v = *reinterpret_cast<const uint4*>(bsm + core_off<KP>(c, k8));
+          const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-          for (int k8 = 0; k8 < G / 8; ++k8) {
-            const uint4 v = *reinterpret_cast<const uint4*>(bsm + core_off<KP>(c, k8));
-            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              // B holds -2c: c = -B/2 exactly
-              const float df0 = xe[k8 * 8 + 2 * i] + 0.5f * bf16_lo(w[i]);
-              const float df1 = xe[k8 * 8 + 2 * i + 1] + 0.5f * bf16_hi(w[i]);
-              d = fmaf(df0, df0, d);
-              d = fmaf(df1, df1, d);
-            }
+          for (int i = 0; i < 4; ++i) {
+            // B holds -2c: c = -B/2 exactly
+            const float df0 = xe[k8 * 8 + 2 * i] + 0.5f * bf16_lo(w[i]);
+            const float df1 = xe[k8 * 8 + 2 * i + 1] + 0.5f * bf16_hi(w[i]);
+            d = fmaf(df0, df0, d);
+            d = fmaf(df1, df1, d);
           }
-          if (d < best) { best = d; bi = c; }
         }
+        return d;
+      };
+      if (refine && !full) {
+        // two candidates: the smaller exact distance, ties to the lower code
+        const int ca = k1 & 0xFF, cb = k2 & 0xFF;
+        const float da = exact_d(ca), db = exact_d(cb);
+        code = (db < da || (db == da && cb < ca)) ? cb : ca;
       }
-      if (refine) code = bi;
+      if (__any_sync(0xffffffffu, full)) {
+        float best = INFINITY;
+        int bi = code;
+#pragma unroll 1
+        for (int cc = 0; cc < kTcCodes / 32; ++cc) {
+          uint32_t r[32];
+          tmem_ld32(t_row + (uint32_t)(cc * 32), r);
+          tmem_wait_ld_tied(r);
+          uint32_t cand = 0;
+#pragma unroll
+          for (int q = 0; q < 32; ++q) cand |= (__uint_as_float(r[q]) <= thr ? 1u : 0u) << q;
+          if (!full) cand = 0;
+          while (cand) {
+            const int c = cc * 32 + __ffs(cand) - 1;
+            cand &= cand - 1;
+            const float d = exact_d(c);
+            if (d < best) { best = d; bi = c; }
+          }
+        }
+        if (full) code = bi;
+      }
     }
     if (ok) p.pool[pool_byte(p.J, p.kind, p.pool_tokens, b, p.H, h, p.tok_off + n, j)] = (uint8_t)code;
     tmem_fence_before();  // TMEM reads ordered before the next tile's barrier and MMA
@@ -385,6 +463,7 @@ bool encode_tc_try(const Geo& g, const void* cb, int kind, const void* x, int64_
   p.Tc = g.Tc; p.H = g.H; p.J = g.J; p.W = g.W; p.kind = kind;
   p.pool = pool; p.tok_off = tok_off; p.pool_tokens = pool_tokens;
   p.faults = faults;
+  p.key_mul = 256u;
   // slot j fastest: the J CTAs of one token chunk run together and share its
   // sectors in L2
   dim3 grid(g.J, (unsigned)ctas_y, g.NB * g.H);
