@@ -18,16 +18,19 @@
 //
 // Epilogue (one thread per sub-vector = one TMEM lane): the row's norm
 // carries a small positive bias (the same for every codeword) that keeps the
-// fast distances positive, so the key "float bits of d with the low 8 bits
-// replaced by the code" orders like d as a signed integer and breaks ties by
-// code; each thread keeps the two smallest keys.  When the two
-// are closer than twice a bound on the fast path's error (plus the 8
-// truncated mantissa bits), the warp re-reads the row from TMEM and the
-// thread re-solves exactly, in fp32 from the differences sum_g (x_g - c_g)^2
-// with a strict "<" in code order, over every codeword whose fast distance is
-// within that bound of the minimum.  The result is the nearest codeword
-// except where two are within fp32 rounding of each other -- the guarantee of
-// the CUDA-core encoder.
+// fast distances positive.  A candidate's key is its fast distance rounded to
+// an integer at a per-row power-of-two scale (23 bits) with the code below
+// it, so keys order like d and break ties by code.  Four chains of sorted
+// key pairs keep each chain's two smallest keys; chain c covers the
+// 8-column groups 32g + 8c.  When the two smallest keys of the row are
+// closer than twice a bound on the fast path's error (plus the keys'
+// rounding), the row is re-solved exactly, in fp32 from the differences
+// sum_g (x_g - c_g)^2, ties to the lower code, over every codeword whose fast
+// distance is within that bound of the minimum: the chain heads within the
+// bound, plus the columns of any chain whose second key is within it (its
+// third is not kept), re-read from TMEM.  The result is the nearest codeword
+// except where two are within fp32 rounding of each other -- the guarantee
+// of the CUDA-core encoder.
 
 #include "common.cuh"
 
@@ -101,6 +104,33 @@ __device__ __forceinline__ void tmem_wait_ld_tied(uint32_t (&r)[32]) {
                  "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]),
                  "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]),
                  "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
+               :
+               : "memory");
+}
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t (&r)[8]) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+               : "r"(taddr)
+               : "memory");
+}
+// Waits for the outstanding TMEM loads, tied to the 64 registers of r.
+__device__ __forceinline__ void tmem_wait_ld_tied64(uint32_t (&r)[8][8]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : "+r"(r[0][0]), "+r"(r[0][1]), "+r"(r[0][2]), "+r"(r[0][3]), "+r"(r[0][4]), "+r"(r[0][5]),
+                 "+r"(r[0][6]), "+r"(r[0][7]), "+r"(r[1][0]), "+r"(r[1][1]), "+r"(r[1][2]), "+r"(r[1][3]),
+                 "+r"(r[1][4]), "+r"(r[1][5]), "+r"(r[1][6]), "+r"(r[1][7]), "+r"(r[2][0]), "+r"(r[2][1]),
+                 "+r"(r[2][2]), "+r"(r[2][3]), "+r"(r[2][4]), "+r"(r[2][5]), "+r"(r[2][6]), "+r"(r[2][7]),
+                 "+r"(r[3][0]), "+r"(r[3][1]), "+r"(r[3][2]), "+r"(r[3][3]), "+r"(r[3][4]), "+r"(r[3][5]),
+                 "+r"(r[3][6]), "+r"(r[3][7])
+               :
+               : "memory");
+  asm volatile(""
+               : "+r"(r[4][0]), "+r"(r[4][1]), "+r"(r[4][2]), "+r"(r[4][3]), "+r"(r[4][4]), "+r"(r[4][5]),
+                 "+r"(r[4][6]), "+r"(r[4][7]), "+r"(r[5][0]), "+r"(r[5][1]), "+r"(r[5][2]), "+r"(r[5][3]),
+                 "+r"(r[5][4]), "+r"(r[5][5]), "+r"(r[5][6]), "+r"(r[5][7]), "+r"(r[6][0]), "+r"(r[6][1]),
+                 "+r"(r[6][2]), "+r"(r[6][3]), "+r"(r[6][4]), "+r"(r[6][5]), "+r"(r[6][6]), "+r"(r[6][7]),
+                 "+r"(r[7][0]), "+r"(r[7][1]), "+r"(r[7][2]), "+r"(r[7][3]), "+r"(r[7][4]), "+r"(r[7][5]),
+                 "+r"(r[7][6]), "+r"(r[7][7])
                :
                : "memory");
 }
@@ -252,10 +282,14 @@ __global__ void __launch_bounds__(kTcThreads, 2) encode_tc_kernel(const EncodeTc
         xx = fmaf(bf16_hi(w[i]), bf16_hi(w[i]), xx);
       }
     }
-    // Fast-path error bound: the fp32 norms and the tensor core's fp32 sums,
-    // each within a few units of 2^-24 of the sum of the terms' magnitudes
-    // (at most 2 (||x||^2 + ||c||^2)); taken as 2^-15 (||x||^2 + max ||c||^2).
-    const float err = 3.0517578e-5f * (xx + nc_max);
+    // Fast-path error bound per codeword.  Every product of two bf16 values is
+    // exact in fp32, so the contraction's error is that of summing its KP
+    // terms: each partial sum is at most S = sum |terms| <= 2 (||x||^2 +
+    // max ||c||^2), and each of the KP - 1 additions rounds (or truncates) by at
+    // most 2^-23 of it, so at most (KP - 1) 2^-22 (||x||^2 + max ||c||^2).  The
+    // fp32 norm ||c||^2 (G fused multiply-adds) adds at most G 2^-24 max ||c||^2;
+    // the norm ||x||^2 is the same for every codeword and cancels.
+    const float err = (float)(4 * (KP - 1) + G) * 5.9604645e-8f * (xx + nc_max);
     // Keys quantize the fast distance at a power-of-two scale sk with
     // d * sk < 2^22 (d <= (|x| + |c|)^2 + 2 err <= 2 (||x||^2 + max ||c||^2) + 2 err):
     // fma(d, sk, 2^23) holds round(d * sk) in its low 23 bits, and
@@ -298,11 +332,12 @@ __global__ void __launch_bounds__(kTcThreads, 2) encode_tc_kernel(const EncodeTc
     phase ^= 1u;
     tmem_fence_after();
 
-    // top-2 keys over the 256 codes, 64 TMEM columns at a time (the next 64
-    // load while these are scanned); 8 independent chains of candidate pairs,
-    // a pair (lo <= hi) merging into a chain's sorted (x1 <= x2) as
-    // x2 = min(max(x1, lo), x2, hi), x1 = min(x1, lo); the code is the key's
-    // low byte (an immediate)
+    // Top-2 keys over the 256 codes, 64 TMEM columns at a time (the next 64
+    // load while these are scanned), in 4 independent chains: chain c takes
+    // the 8-column groups 32g + 8c (g = 0..7), so that its 64 columns can be
+    // re-read with eight 8-column loads.  A pair (lo <= hi) merges into a
+    // chain's sorted (x1 <= x2) as x2 = min(max(x1, lo), x2, hi),
+    // x1 = min(x1, lo); the code is the key's low byte (an immediate).
     auto qkey = [&](uint32_t v, uint32_t code) -> int {
       const float y = __fmaf_rn(__uint_as_float(v), sk, 8388608.f);
       return (int)(__float_as_uint(y) * p.key_mul + code);
@@ -329,7 +364,7 @@ __global__ void __launch_bounds__(kTcThreads, 2) encode_tc_kernel(const EncodeTc
         const int k0 = qkey(cur[col >> 5][col & 31], (uint32_t)(64 * i + col));
         const int k1v = qkey(cur[(col + 1) >> 5][(col + 1) & 31], (uint32_t)(64 * i + col + 1));
         const int lo = min(k0, k1v), hi = max(k0, k1v);
-        const int c = pp & 3;
+        const int c = (pp >> 2) & 3;
         x2[c] = min(min(max(x1[c], lo), x2[c]), hi);
         x1[c] = min(x1[c], lo);
       }
@@ -345,30 +380,23 @@ __global__ void __launch_bounds__(kTcThreads, 2) encode_tc_kernel(const EncodeTc
 #pragma unroll
     for (int c = 0; c < 4; ++c) k2 = min(k2, x1[c] != k1 ? x1[c] : 0x7FFFFFFF);
     int code = k1 & 0xFF;
-    // the gap of the two smallest keys in units of 1/sk; each key rounds by
-    // at most half a unit
-    const float gap = (float)((k2 >> 8) - (k1 >> 8));
-    const bool refine = ok && !(gap > 2.f * err * sk + 2.f);
+    // a key is a candidate when its gap to k1 (units of 1/sk) is within twice
+    // the fast path's error bound plus the keys' rounding (half a unit each)
+    const float bound = 2.f * err * sk + 2.f;
+    auto near = [&](int k) -> bool { return !((float)((k >> 8) - (k1 >> 8)) > bound); };
+    const bool refine = ok && near(k2);
     if (__any_sync(0xffffffffu, refine)) {
-      // Only the codes whose fast distance is within 2 err of the minimum can
-      // be the nearest.  The third smallest chain value is the row's third
-      // smallest key unless the two smallest share a chain (then k2 is that
-      // chain's second); when it is farther than the bound from k1, the two
-      // codes of k1 and k2 are the only candidates and are solved directly,
-      // otherwise the row is scanned in full.
-      bool full = false;
+      // Only codes whose fast distance is within 2 err of the minimum can be
+      // the nearest.  The sorted chain values are the row's smallest keys up
+      // to the first chain second within the bound (that chain's third is not
+      // kept), so the candidates are the chain heads within the bound plus
+      // every column of the chains whose second is within it, re-read from
+      // TMEM.
+      uint32_t rescan = 0;
       if (refine) {
-        bool same = false;
-        int k3 = 0x7FFFFFFF;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          same |= x2[c] == k2;
-          k3 = min(k3, x1[c] > k2 ? x1[c] : 0x7FFFFFFF);
-          k3 = min(k3, x2[c] > k2 ? x2[c] : 0x7FFFFFFF);
-        }
-        full = same || !((float)((k3 >> 8) - (k1 >> 8)) > 2.f * err * sk + 2.f);
+        for (int c = 0; c < 4; ++c) rescan |= near(x2[c]) ? 1u << c : 0u;
       }
-      const float thr = (float)(k1 >> 8) * inv_sk + 2.f * err + 2.f * inv_sk;
       float xe[G];
 #pragma unroll
       for (int k8 = 0; k8 < G / 8; ++k8) {
@@ -395,33 +423,40 @@ __global__ void __launch_bounds__(kTcThreads, 2) encode_tc_kernel(const EncodeTc
         }
         return d;
       };
-      if (refine && !full) {
-        // two candidates: the smaller exact distance, ties to the lower code
-        const int ca = k1 & 0xFF, cb = k2 & 0xFF;
-        const float da = exact_d(ca), db = exact_d(cb);
-        code = (db < da || (db == da && cb < ca)) ? cb : ca;
-      }
-      if (__any_sync(0xffffffffu, full)) {
-        float best = INFINITY;
-        int bi = code;
+      // the smallest exact distance, ties to the lower code
+      float best = INFINITY;
+      int bi = code;
+      auto consider = [&](int c) {
+        const float d = exact_d(c);
+        if (d < best || (d == best && c < bi)) { best = d; bi = c; }
+      };
+      if (refine) {
 #pragma unroll 1
-        for (int cc = 0; cc < kTcCodes / 32; ++cc) {
-          uint32_t r[32];
-          tmem_ld32(t_row + (uint32_t)(cc * 32), r);
-          tmem_wait_ld_tied(r);
-          uint32_t cand = 0;
-#pragma unroll
-          for (int q = 0; q < 32; ++q) cand |= (__uint_as_float(r[q]) <= thr ? 1u : 0u) << q;
-          if (!full) cand = 0;
-          while (cand) {
-            const int c = cc * 32 + __ffs(cand) - 1;
-            cand &= cand - 1;
-            const float d = exact_d(c);
-            if (d < best) { best = d; bi = c; }
-          }
-        }
-        if (full) code = bi;
+        for (int c = 0; c < 4; ++c)
+          if (!(rescan >> c & 1u) && near(x1[c])) consider(x1[c] & 0xFF);
       }
+      const float thr = (float)(k1 >> 8) * inv_sk + 2.f * err + 2.f * inv_sk;
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        if (!__any_sync(0xffffffffu, rescan >> c & 1u)) continue;
+        uint32_t r[8][8];
+#pragma unroll
+        for (int g = 0; g < 8; ++g) tmem_ld8(t_row + (uint32_t)(32 * g + 8 * c), r[g]);
+        tmem_wait_ld_tied64(r);
+        uint64_t cand = 0;
+#pragma unroll
+        for (int g = 0; g < 8; ++g) {
+#pragma unroll
+          for (int q = 0; q < 8; ++q) cand |= (uint64_t)(__uint_as_float(r[g][q]) <= thr ? 1u : 0u) << (8 * g + q);
+        }
+        if (!(rescan >> c & 1u)) cand = 0;
+        while (cand) {
+          const int bit = __ffsll((long long)cand) - 1;
+          cand &= cand - 1;
+          consider(32 * (bit >> 3) + 8 * c + (bit & 7));
+        }
+      }
+      if (refine) code = bi;
     }
     if (ok) p.pool[pool_byte(p.J, p.kind, p.pool_tokens, b, p.H, h, p.tok_off + n, j)] = (uint8_t)code;
     tmem_fence_before();  // TMEM reads ordered before the next tile's barrier and MMA
