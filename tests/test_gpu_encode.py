@@ -236,6 +236,44 @@ def test_tensor_core_encode_exact_ties_go_to_lowest_index():
     assert _accept(Xe, cb, tc, g) == 0
 
 
+def test_tensor_core_encode_near_tie_clusters():
+    """Near-duplicate codewords (one element one bf16 step apart) and
+    sub-vectors drawn tightly around them: nearly every row's two best fast
+    distances fall within the fast path's error bound, so the rows are
+    re-solved exactly.  The clusters sit in different top-2 chains (codes 16
+    and 40; chains take the code groups (code % 32) // 8), in one chain (24
+    and 30) and as a triple over two chains (64, 72 and 65), so both the
+    two-head re-solve and the chain re-read run.  Every code must be the
+    oracle's nearest, and both members of each cluster must win somewhere."""
+    L = _L()
+    T, N, H, D, tc, G = 4, 768, 1, 128, 4, 16
+    W, J = G // tc, D * tc // G
+    X = synth.loop_correlated(seed=72, n_loop=T, n_tokens=N, n_heads=H, head_dim=D)
+    cb = synth.codebook_from_rows(X, tc, G, 256, seed=73)
+
+    def nudge(v, e):   # element e of every [tc][W] codeword one bf16 step up in magnitude
+        f = np.ascontiguousarray(v, dtype=np.float32).reshape(v.shape[:-2] + (tc * W,)).copy()
+        f.view(np.uint32)[..., e] += 0x10000
+        return f.reshape(v.shape)
+
+    for c0, dups in {16: [(40, 0)], 24: [(30, 1)], 64: [(72, 2), (65, 3)]}.items():
+        for cd, e in dups:
+            cb[:, :, :, cd] = nudge(cb[:, :, :, c0], e)
+    rng = np.random.default_rng(74)
+    sel = np.array([16, 24, 64])[np.arange(N) % 3]
+    cs = cb[0, 0][:, sel]                       # [J][N][tc][W]
+    Xe = np.empty_like(X)
+    for t in range(tc):
+        Xe[t, :, 0, :] = cs[:, :, t, :].transpose(1, 0, 2).reshape(N, J * W)
+    Xe = synth.round_bf16(Xe + 0.006 * rng.standard_normal(Xe.shape).astype(np.float32))
+    desc = L.make_desc(T, tc, H, D, G, 256)
+    g, _ = _encode_gpu(desc, cb, Xe, L.LOOPVQ_KEYS, N)
+    idx, _, _ = O.encode(Xe, cb, tc)
+    for c in (16, 40, 24, 30, 64, 72, 65):
+        assert (idx == c).any() and (g == c).any(), c
+    assert _accept(Xe, cb, tc, g) == 0
+
+
 @pytest.mark.parametrize("n", [1, 8, 200])
 @pytest.mark.parametrize("tc,G", [(4, 16), (4, 32), (4, 64), (2, 8), (1, 4)])
 @pytest.mark.parametrize("xdt", ["bf16", "f32"])
