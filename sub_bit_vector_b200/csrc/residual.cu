@@ -21,10 +21,17 @@
 //   value params  [T][H][pool_tokens][D/32] half2 (min, scale)
 //
 // Decode at loop step t streams tiles of the t+1 residual planes into shared
-// memory by bulk copies, rebuilds each token's key and value rows from them
-// (added in step order, as the encoder did; eight lanes per token, each with
-// D/8 channels) and runs split-K attention with an fp32 online softmax; the
-// last split of a (request, head) merges the splits.
+// memory by bulk copies (eight lanes per token, each with D/8 channels) and
+// runs split-K attention with an fp32 online softmax; the last split of a
+// (request, head) merges the splits.  The rebuilt key is min + code * scale
+// summed over the planes, so the score q . K is
+//   sum_d q_d sum_p min_p[d]  +  sum_p sum_d (q_d scale_p[d]) code_p[d]:
+// from two planes on, the 8 warps sharing a key group turn q_d scale_p[d] into
+// three int8 digits per channel block (under the block's own scale) once per
+// tile, and each lane sums its block with dp4a over its codes expanded to
+// bytes; with one plane the key row is rebuilt per element as the encoder
+// did.  Values fold the same way: the weighted sum takes code * scale per
+// element and the planes' minima once per token.
 
 #include <cuda_fp16.h>
 #include <math.h>
@@ -194,8 +201,8 @@ struct ResConsumerSync {
   __device__ __forceinline__ void operator()() const { asm volatile("bar.sync 1, %0;" ::"n"(kRW * 32) : "memory"); }
 };
 
-template <int CPL>
-__global__ void __launch_bounds__(kRThreads) res_decode_kernel(const ResDecParams p) {
+template <int CPL, bool kIntKeys>
+__global__ void __launch_bounds__(kRThreads, 1) res_decode_kernel(const ResDecParams p) {
   constexpr int D = CPL * kRLanesPerTok;
   extern __shared__ __align__(128) uint8_t rsm[];
   __shared__ float wpart[kRW][D + 2];
@@ -277,26 +284,78 @@ __global__ void __launch_bounds__(kRThreads) res_decode_kernel(const ResDecParam
 
   // consumers
   const int grp = lane / kRLanesPerTok, li = lane % kRLanesPerTok;
-  float qv[CPL];
-#pragma unroll
-  for (int i = 0; i < CPL; ++i) {
-    const size_t qi = unit * D + li * CPL + i;
-    qv[i] = (p.q_bf16 ? __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(p.q)[qi])
-                      : reinterpret_cast<const float*>(p.q)[qi]) *
+  // The query row in log2 units, for the key-digit passes.
+  float* const qs = reinterpret_cast<float*>(rsm + (size_t)NS * stage_bytes);
+  int8_t* const dig = reinterpret_cast<int8_t*>(qs + D);  // [2 tile parities][2 key groups][planes][3][D]
+  __shared__ float kred[2][2][8][2];                       // per parity, group, warp: max |W|, partial C
+  for (int d = tid; d < D; d += kRW * 32)
+    qs[d] = (p.q_bf16 ? __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(p.q)[unit * D + d])
+                      : reinterpret_cast<const float*>(p.q)[unit * D + d]) *
             p.scale_log2;
-  }
+  ResConsumerSync{}();
+  float qv[CPL];  // the per-element key path's query channels li*CPL.. (log2 units)
+#pragma unroll
+  for (int c = 0; c < CPL; ++c) qv[c] = qs[li * CPL + c];
   float m = -INFINITY, l = 0.f, o[CPL];
 #pragma unroll
   for (int i = 0; i < CPL; ++i) o[i] = 0.f;
   const int j = warp * kRTokPerWarp + grp;  // token of the tile
+  const int gi = warp >> 3;                 // its key group within the tile (tokens 32 gi ..)
+  const int ht = (warp & 7) * 32 + lane;    // thread index among the 8 warps of that group
   for (int i = 0; i < n_tiles; ++i) {
     const int st = i % NS;
     if (!mbar_wait_bounded(smem_u32(full + st), (i / NS) & 1)) set_fault(p.status, LOOPVQ_FAULT_TIMEOUT);
     const int n = min(kRTile, t1 - (t0 + i * kRTile));
     const uint8_t* sb = rsm + (size_t)st * stage_bytes;
-    float k[CPL], v[CPL];
+    const int par = i & 1;
+    // ---- key digits of this tile's group: the score of token n is
+    //   C + sum_p sum_d W_p[d] code_p[n][d],  W_p[d] = q[d] * scale_p[g][d],
+    //   C = sum_d q[d] sum_p min_p[g][d].
+    // Warp hw of the group's 8 writes channel block hw (the block lane hw of a
+    // token scores): W over all planes as sigma (w0 + w1 / 128 + w2 / 16384)
+    // with int8 digits, sigma = the block's max |W| / 127, so that the sum over
+    // the block's channels runs as integer dot products.  Bytes are laid out as
+    // a lane expands its codes (even nibbles, then odd ones, per 8 channels).
+    if constexpr (kIntKeys) {
+      const int hw = warp & 7;
+      float amax = 0.f, cpart = 0.f;
+      for (int e = lane; e < planes * CPL; e += 32) {
+        const int s = e / CPL, d = hw * CPL + (e - s * CPL);
+        const float2 kpar = __half22float2(*reinterpret_cast<const __half2*>(sb + (size_t)s * pb + 72 * D + (gi * D + d) * 4));
+        amax = fmaxf(amax, fabsf(qs[d] * kpar.y));
+        cpart = fmaf(qs[d], kpar.x, cpart);
+      }
 #pragma unroll
-    for (int c = 0; c < CPL; ++c) k[c] = v[c] = 0.f;
+      for (int x = 16; x >= 1; x >>= 1) {
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, x));
+        cpart += __shfl_xor_sync(0xffffffffu, cpart, x);
+      }
+      const float inv = amax > 0.f ? 127.f / amax : 0.f;
+      for (int e = lane; e < planes * CPL; e += 32) {
+        const int s = e / CPL, mm = e - s * CPL, d = hw * CPL + mm;
+        const float2 kpar = __half22float2(*reinterpret_cast<const __half2*>(sb + (size_t)s * pb + 72 * D + (gi * D + d) * 4));
+        const float r0 = qs[d] * kpar.y * inv;
+        const float w0 = rintf(r0);
+        const float r1 = (r0 - w0) * 128.f;
+        const float w1 = rintf(r1);
+        const float w2 = rintf((r1 - w1) * 128.f);
+        const int pos = (hw * (CPL / 4) + (((mm >> 3) << 1) | (mm & 1))) * 4 + ((mm & 7) >> 1);
+        int8_t* db = dig + ((size_t)((par * 2 + gi) * planes + s) * 3) * D + pos;
+        db[0] = (int8_t)w0;
+        db[D] = (int8_t)w1;
+        db[2 * D] = (int8_t)w2;
+      }
+      if (lane == 0) { kred[par][gi][hw][0] = amax; kred[par][gi][hw][1] = cpart; }
+      asm volatile("bar.sync %0, 256;" ::"r"(2 + gi) : "memory");
+    }
+    float v[CPL];
+#pragma unroll
+    for (int c = 0; c < CPL; ++c) v[c] = 0.f;
+    int acc0 = 0, acc1 = 0, acc2 = 0;
+    float k[CPL];     // the per-element key path: the token's reconstructed key channels
+#pragma unroll
+    for (int c = 0; c < CPL; ++c) k[c] = 0.f;
+    float vlo = 0.f;  // the planes' value minima of this lane's group, added once
     for (int s = 0; s < planes; ++s) {
       const uint8_t* pl = sb + (size_t)s * pb;
       uint32_t kc[CPL / 8], vc[CPL / 8];
@@ -308,29 +367,72 @@ __global__ void __launch_bounds__(kRThreads) res_decode_kernel(const ResDecParam
         kc[0] = *reinterpret_cast<const uint32_t*>(pl + j * (D / 2) + li * 4);
         vc[0] = *reinterpret_cast<const uint32_t*>(pl + 32 * D + j * (D / 2) + li * 4);
       }
-      const float2 vpar =
-          __half22float2(*reinterpret_cast<const __half2*>(pl + 64 * D + (j * (D / kRG) + (li * CPL) / kRG) * 4));
-      const uint4* kp = reinterpret_cast<const uint4*>(pl + 72 * D + ((j / kRG) * D + li * CPL) * 4);
+      if constexpr (kIntKeys) {
+        // codes as bytes: word 2x holds the even nibbles of code word x, 2x + 1 the odd ones
+        uint32_t bw[CPL / 4];
+  #pragma unroll
+        for (int x = 0; x < CPL / 8; ++x) { bw[2 * x] = kc[x] & 0x0F0F0F0Fu; bw[2 * x + 1] = (kc[x] >> 4) & 0x0F0F0F0Fu; }
+        const int8_t* db = dig + ((size_t)((par * 2 + gi) * planes + s) * 3) * D + li * CPL;
+        uint32_t dw[3][CPL / 4];
+  #pragma unroll
+        for (int k = 0; k < 3; ++k) {
+          if constexpr (CPL == 16) {
+            const uint4 t4 = *reinterpret_cast<const uint4*>(db + k * D);
+            dw[k][0] = t4.x; dw[k][1] = t4.y; dw[k][2] = t4.z; dw[k][3] = t4.w;
+          } else {
+            const uint2 t2 = *reinterpret_cast<const uint2*>(db + k * D);
+            dw[k][0] = t2.x; dw[k][1] = t2.y;
+          }
+        }
+  #pragma unroll
+        for (int x = 0; x < CPL / 4; ++x) {
+          asm("dp4a.u32.s32 %0, %1, %2, %0;" : "+r"(acc0) : "r"(bw[x]), "r"(dw[0][x]));
+          asm("dp4a.u32.s32 %0, %1, %2, %0;" : "+r"(acc1) : "r"(bw[x]), "r"(dw[1][x]));
+          asm("dp4a.u32.s32 %0, %1, %2, %0;" : "+r"(acc2) : "r"(bw[x]), "r"(dw[2][x]));
+        }
+      } else {
+        // one step's residual plane: rebuild the key channels in step order
+        const uint4* kp = reinterpret_cast<const uint4*>(pl + 72 * D + ((j / kRG) * D + li * CPL) * 4);
 #pragma unroll
-      for (int w = 0; w < CPL / 4; ++w) {
-        const uint4 pw = kp[w];
-        const uint32_t pr[4] = {pw.x, pw.y, pw.z, pw.w};
+        for (int w = 0; w < CPL / 4; ++w) {
+          const uint4 pw = kp[w];
+          const uint32_t pr[4] = {pw.x, pw.y, pw.z, pw.w};
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int c = w * 4 + u;
-          const float2 kpar = __half22float2(*reinterpret_cast<const __half2*>(&pr[u]));
-          k[c] = __fadd_rn(k[c], dq4((kc[c >> 3] >> (4 * (c & 7))) & 15u, kpar.x, kpar.y));
-          v[c] = __fadd_rn(v[c], dq4((vc[c >> 3] >> (4 * (c & 7))) & 15u, vpar.x, vpar.y));
+          for (int u = 0; u < 4; ++u) {
+            const int c = w * 4 + u;
+            const float2 kpar = __half22float2(*reinterpret_cast<const __half2*>(&pr[u]));
+            k[c] = __fadd_rn(k[c], dq4((kc[c >> 3] >> (4 * (c & 7))) & 15u, kpar.x, kpar.y));
+          }
         }
       }
+      const float2 vpar =
+          __half22float2(*reinterpret_cast<const __half2*>(pl + 64 * D + (j * (D / kRG) + (li * CPL) / kRG) * 4));
+      vlo += vpar.x;
+#pragma unroll
+      for (int c = 0; c < CPL; ++c) v[c] = fmaf((float)((vc[c >> 3] >> (4 * (c & 7))) & 15u), vpar.y, v[c]);
     }
+#pragma unroll
+    for (int c = 0; c < CPL; ++c) v[c] += vlo;
     __syncwarp();
     if (lane == 0) mbar_arrive(smem_u32(empty + st));  // the warp's reads of this stage are done
-    float a = 0.f;
+    float a;
+    if constexpr (kIntKeys) {
+      // this lane's block: sigma_li (w0 + w1 / 128 + w2 / 16384) summed by dp4a
+      a = ((float)acc0 + (float)acc1 * (1.f / 128.f) + (float)acc2 * (1.f / 16384.f)) *
+          (kred[par][gi][li][0] * (1.f / 127.f));
 #pragma unroll
-    for (int c = 0; c < CPL; ++c) a = fmaf(qv[c], k[c], a);
+      for (int x = kRLanesPerTok / 2; x >= 1; x >>= 1) a += __shfl_xor_sync(0xffffffffu, a, x);
+      float csum = 0.f;
 #pragma unroll
-    for (int x = kRLanesPerTok / 2; x >= 1; x >>= 1) a += __shfl_xor_sync(0xffffffffu, a, x);
+      for (int w = 0; w < 8; ++w) csum += kred[par][gi][w][1];
+      a += csum;
+    } else {
+      a = 0.f;
+#pragma unroll
+      for (int c = 0; c < CPL; ++c) a = fmaf(qv[c], k[c], a);
+#pragma unroll
+      for (int x = kRLanesPerTok / 2; x >= 1; x >>= 1) a += __shfl_xor_sync(0xffffffffu, a, x);
+    }
     const float sc = j < n ? a : -INFINITY;
     const float mn = fmaxf(m, sc);
     if (mn != -INFINITY) {
@@ -503,23 +605,22 @@ extern "C" loopvq_status loopvq_residual_decode_attn(const loopvq_residual_desc*
   p.tickets = (uint32_t*)((uint8_t*)workspace + ws.tickets_off);
   p.partials = (float*)((uint8_t*)workspace + ws.partials_off);
   const int stage_bytes = (loop_step + 1) * res_plane_bytes(g.D);
-  int ns = kRSmemBudget / stage_bytes;
+  // after the stages: the query row (D floats) and the key digits
+  // (2 tile parities x 2 key groups x planes x 3 digits x D bytes)
+  const int extra = g.D * 4 + 12 * (loop_step + 1) * g.D;
+  int ns = (kRSmemBudget - extra) / stage_bytes;
   if (ns > kRMaxStages) ns = kRMaxStages;
   if (ns < 1) return LOOPVQ_ERR_UNSUPPORTED;   // more planes than one stage can hold
   p.n_stages = ns;
-  const size_t smem = (size_t)ns * stage_bytes;
+  const size_t smem = (size_t)ns * stage_bytes + extra;
   dim3 grid(ms, g.Hq, batch);
   cudaStream_t s = (cudaStream_t)stream;
-  if (g.D == 128) {
-    if (cudaFuncSetAttribute(res_decode_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-        cudaSuccess)
-      return LOOPVQ_ERR_CUDA;
-    res_decode_kernel<16><<<grid, kRThreads, smem, s>>>(p);
-  } else {
-    if (cudaFuncSetAttribute(res_decode_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-        cudaSuccess)
-      return LOOPVQ_ERR_CUDA;
-    res_decode_kernel<8><<<grid, kRThreads, smem, s>>>(p);
-  }
+  // integer key scores from two planes on; one plane keeps the per-element path
+  const bool int_keys = loop_step >= 1;
+  auto kfn = g.D == 128 ? (int_keys ? res_decode_kernel<16, true> : res_decode_kernel<16, false>)
+                        : (int_keys ? res_decode_kernel<8, true> : res_decode_kernel<8, false>);
+  if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    return LOOPVQ_ERR_CUDA;
+  kfn<<<grid, kRThreads, smem, s>>>(p);
   return cudaGetLastError() == cudaSuccess ? LOOPVQ_OK : LOOPVQ_ERR_CUDA;
 }
