@@ -65,6 +65,16 @@ __device__ __forceinline__ uint32_t q4(float x, float lo, float sc) {
   return (uint32_t)fminf(fmaxf(v, 0.f), 15.f);
 }
 __device__ __forceinline__ float dq4(uint32_t q, float lo, float sc) { return __fadd_rn(lo, __fmul_rn((float)q, sc)); }
+// Exact float of nibble i (0..7) of x, given x12 = x >> 12: nibbles 0..4 are
+// read in place and 5..7 from x12 (slots 2..4).  The nibble at slot s is
+// OR-ed into the mantissa of 2^(23 - 4s), whose last place at bit 4s is worth
+// 1, so subtracting 2^(23 - 4s) leaves it exactly (no integer conversion).
+__device__ __forceinline__ float nibf(uint32_t x, uint32_t x12, int i) {
+  const int s = i <= 4 ? i : i - 3;
+  const uint32_t src = i <= 4 ? x : x12;
+  const uint32_t ebits = (uint32_t)(150 - 4 * s) << 23;
+  return __fsub_rn(__uint_as_float((src & (0xFu << (4 * s))) | ebits), __uint_as_float(ebits));
+}
 
 struct ResEncParams {
   const void* x;
@@ -392,6 +402,9 @@ __global__ void __launch_bounds__(kRThreads, 1) res_decode_kernel(const ResDecPa
         }
       } else {
         // one step's residual plane: rebuild the key channels in step order
+        uint32_t kc12[CPL / 8];
+#pragma unroll
+        for (int x = 0; x < CPL / 8; ++x) kc12[x] = kc[x] >> 12;
         const uint4* kp = reinterpret_cast<const uint4*>(pl + 72 * D + ((j / kRG) * D + li * CPL) * 4);
 #pragma unroll
         for (int w = 0; w < CPL / 4; ++w) {
@@ -401,15 +414,18 @@ __global__ void __launch_bounds__(kRThreads, 1) res_decode_kernel(const ResDecPa
           for (int u = 0; u < 4; ++u) {
             const int c = w * 4 + u;
             const float2 kpar = __half22float2(*reinterpret_cast<const __half2*>(&pr[u]));
-            k[c] = __fadd_rn(k[c], dq4((kc[c >> 3] >> (4 * (c & 7))) & 15u, kpar.x, kpar.y));
+            k[c] = __fadd_rn(k[c], __fadd_rn(kpar.x, __fmul_rn(nibf(kc[c >> 3], kc12[c >> 3], c & 7), kpar.y)));
           }
         }
       }
       const float2 vpar =
           __half22float2(*reinterpret_cast<const __half2*>(pl + 64 * D + (j * (D / kRG) + (li * CPL) / kRG) * 4));
       vlo += vpar.x;
+      uint32_t vc12[CPL / 8];
 #pragma unroll
-      for (int c = 0; c < CPL; ++c) v[c] = fmaf((float)((vc[c >> 3] >> (4 * (c & 7))) & 15u), vpar.y, v[c]);
+      for (int x = 0; x < CPL / 8; ++x) vc12[x] = vc[x] >> 12;
+#pragma unroll
+      for (int c = 0; c < CPL; ++c) v[c] = fmaf(nibf(vc[c >> 3], vc12[c >> 3], c & 7), vpar.y, v[c]);
     }
 #pragma unroll
     for (int c = 0; c < CPL; ++c) v[c] += vlo;
