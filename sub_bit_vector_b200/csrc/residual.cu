@@ -174,8 +174,9 @@ __global__ void __launch_bounds__(256) res_encode_values(const ResEncParams p) {
 // 64 tokens -- for every plane s <= t the tile's key codes, value codes, value
 // parameters and key parameters -- with bulk copies (no multicast) into a
 // ring of shared-memory stages; 16 consumer warps take one token per group of
-// eight lanes (lane i of a group owns channels i*D/8 ..), rebuild the rows
-// from the staged planes in step order and keep an fp32 online softmax.
+// eight lanes (lane i of a group owns channels i*D/8 ..), score it from the
+// staged planes (integer key digits from two planes on, the rebuilt key row
+// with one plane) and keep an fp32 online softmax.
 constexpr int kRW = 16;                       // consumer warps
 constexpr int kRThreads = (kRW + 1) * 32;     // + the producer warp
 constexpr int kRLanesPerTok = 8;
