@@ -71,9 +71,14 @@ def test_residual_encode_bit_exact(N, H, D, dtype, kind):
     np.testing.assert_array_equal(got_sc.view(np.uint16), ref_sc.view(np.uint16))
 
 
-def test_residual_decode_matches_oracle_every_step():
+@pytest.mark.parametrize("T,D", [(4, 128), (6, 64)])
+def test_residual_decode_matches_oracle_every_step(T, D):
+    """Every loop step against the oracle: step 0 rebuilds the key row per
+    element, later steps score keys with integer digits (D = 128 and D = 64
+    instances, up to 6 planes), ragged contexts with a one-token last tile,
+    GQA 2."""
     L = _L()
-    T, H, Hq, D = 4, 2, 4, 128
+    H, Hq = 2, 4
     ctx = [3000, 301, 45, 1, 0]
     pool = sum(-(-max(c, 1) // 32) * 32 for c in ctx)
     offs = np.cumsum([0] + [-(-max(c, 1) // 32) * 32 for c in ctx])[:-1]
