@@ -523,9 +523,16 @@ LOOPVQ_API size_t loopvq_residual_decode_workspace_bytes(const loopvq_residual_d
 /*
  * Decode attention at loop step t over the residual-coded cache: request r's
  * ctx_len[r] tokens at pool positions tok_off[r] .. (every token coded, no
- * bf16 window); each token's key and value rows are rebuilt from the t+1
- * residual planes added in step order (the encoder's reconstruction, bit
- * for bit) and o = softmax(softmax_scale * q . k) v in fp32.
+ * bf16 window); o = softmax(softmax_scale * q . k) v in fp32 over the key and
+ * value rows that the t+1 residual planes rebuild (the encoder's
+ * reconstruction).  At t = 0 the key row is rebuilt per element as the
+ * encoder does; from t = 1 on q . k is taken as sum_d q_d sum_p min_p[d] plus
+ * integer dot products of the codes with q_d scale_p[d] in three int8 digits
+ * per 16-channel block (relative error below 2.5e-7 of the block's largest
+ * weight), and values as code * scale per element plus the minima once per
+ * token.  The t+1 planes of a 64-token tile must fit one shared-memory
+ * stage: t+1 <= 16 at D = 128, <= 33 at D = 64 (LOOPVQ_ERR_UNSUPPORTED
+ * beyond).
  *   ctx_len, tok_off : device [batch] int32 / int64.
  *   q [batch][Hq][D] in q_dtype; out [batch][Hq][D] fp32; lse_out nullable.
  *   codesK/V  : 8-byte aligned; paramsK 16-byte, paramsV 4-byte aligned.
