@@ -144,3 +144,41 @@ def test_residual_beats_per_step_coding_on_gpu_codes():
             u = _unpack(desc1, c1, p1, kind, 0, N, N)
             err_ind += np.mean((O.residual_reconstruct(*u, "k" if kind == 0 else "v", 0) - X[t]) ** 2)
         assert err_res < err_ind, (kind, err_res, err_ind)
+
+
+def test_residual_decode_most_planes_and_refusal_beyond():
+    """16 planes (loop step 15) are the most a 64-token tile stage holds at
+    D = 128 next to the key digits: that launch matches the oracle; loop step
+    16 is refused before anything is launched (the buffers are real and in
+    range all the same)."""
+    L = _L()
+    T, H, D, c = 17, 1, 128, 40
+    pool = 64
+    desc = L.make_residual_desc(T, H, D)
+    ck = torch.zeros(L.loopvq_residual_codes_bytes(desc, pool), dtype=torch.uint8, device="cuda")
+    cv = torch.zeros_like(ck)
+    pk = torch.zeros(L.loopvq_residual_params_bytes(desc, 0, pool) // 2, dtype=torch.float16, device="cuda")
+    pv = torch.zeros(L.loopvq_residual_params_bytes(desc, 1, pool) // 2, dtype=torch.float16, device="cuda")
+    K = synth.loop_correlated(seed=970, n_loop=T, n_tokens=c, n_heads=H, head_dim=D, n_outlier=4)
+    V = synth.loop_correlated(seed=971, n_loop=T, n_tokens=c, n_heads=H, head_dim=D)
+    for kind, X, cc, pp in ((0, K, ck, pk), (1, V, cv, pv)):
+        x = torch.from_numpy(np.ascontiguousarray(X, dtype=np.float32)).cuda().to(torch.bfloat16)
+        L.loopvq_residual_encode(desc, kind, x, c, c * H * D, H * D, D, cc, pp, 0, pool)
+    (kc, kl, ks), (vc, vl, vs) = (O.residual_encode(np.asarray(K, dtype=np.float32), "k")[:3],
+                                  O.residual_encode(np.asarray(V, dtype=np.float32), "v")[:3])
+    ctx_d = torch.tensor([c], dtype=torch.int32, device="cuda")
+    off_d = torch.zeros(1, dtype=torch.int64, device="cuda")
+    ws = torch.zeros(L.loopvq_residual_decode_workspace_bytes(desc, 1, c), dtype=torch.uint8, device="cuda")
+    out = torch.zeros((1, H, D), dtype=torch.float32, device="cuda")
+    q = synth.round_bf16(np.random.default_rng(972).standard_normal((1, H, D)).astype(np.float32))
+    qd = torch.from_numpy(q).cuda().to(torch.bfloat16)
+    L.loopvq_residual_decode_attn(desc, 1, c, ctx_d, off_d, pool, ck, pk, cv, pv, qd, 15, D ** -0.5, out, None, ws)
+    torch.cuda.synchronize()
+    o_ref, _ = O.residual_decode_attention(q[0], 15, kc, kl, ks, vc, vl, vs, D ** -0.5)
+    e = np.max(np.abs(out.cpu().numpy()[0, 0] - o_ref[0])) / np.max(np.abs(o_ref[0]))
+    assert e <= TOL, e
+    with pytest.raises(L.LoopVQError) as err:
+        L.loopvq_residual_decode_attn(desc, 1, c, ctx_d, off_d, pool, ck, pk, cv, pv, qd, 16, D ** -0.5, out, None,
+                                      ws)
+    assert err.value.status == L.LOOPVQ_ERR_UNSUPPORTED
+    assert L.loopvq_read_device_status(ws)[1] == 0
