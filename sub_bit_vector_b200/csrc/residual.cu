@@ -312,7 +312,6 @@ __global__ void __launch_bounds__(kRThreads, 1) res_decode_kernel(const ResDecPa
   for (int i = 0; i < CPL; ++i) o[i] = 0.f;
   const int j = warp * kRTokPerWarp + grp;  // token of the tile
   const int gi = warp >> 3;                 // its key group within the tile (tokens 32 gi ..)
-  const int ht = (warp & 7) * 32 + lane;    // thread index among the 8 warps of that group
   for (int i = 0; i < n_tiles; ++i) {
     const int st = i % NS;
     if (!mbar_wait_bounded(smem_u32(full + st), (i / NS) & 1)) set_fault(p.status, LOOPVQ_FAULT_TIMEOUT);
@@ -357,6 +356,9 @@ __global__ void __launch_bounds__(kRThreads, 1) res_decode_kernel(const ResDecPa
         db[2 * D] = (int8_t)w2;
       }
       if (lane == 0) { kred[par][gi][hw][0] = amax; kred[par][gi][hw][1] = cpart; }
+      // the group's 8 warps (named barrier 2 + gi): every block's digits and
+      // scale are written before any lane reads them; the tile parity keeps
+      // the next tile's writes off what a slower warp may still be reading
       asm volatile("bar.sync %0, 256;" ::"r"(2 + gi) : "memory");
     }
     float v[CPL];
