@@ -141,35 +141,52 @@ __global__ void __launch_bounds__(kREncWarps * 32, 4) res_encode_keys(const ResE
   }
 }
 
-// Values: one warp per (token, head, 32-channel group); lane = channel, the
-// group's min and max by shuffles.
+// Values: one warp per (two tokens, head, 32-channel group); lane = channel,
+// each group's min and max by shuffles.  The two tokens' step chains are
+// independent and interleave (1.15 vs 1.30 ms per 32K x 16 x 128 x 4 tensor
+// with one token per warp, the same codes and parameters; four or eight
+// tokens per warp lose more to registers than they gain).
 __global__ void __launch_bounds__(256) res_encode_values(const ResEncParams p) {
   const int lane = threadIdx.x & 31;
   const int64_t wid = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int cgroups = p.D / kRG;
-  if (wid >= p.n_tokens * p.H * cgroups) return;
+  const int64_t n_pairs = (p.n_tokens + 1) / 2;
+  if (wid >= n_pairs * p.H * cgroups) return;
   const int cg = (int)(wid % cgroups);
   const int h = (int)((wid / cgroups) % p.H);
-  const int64_t n = wid / ((int64_t)cgroups * p.H);
+  const int64_t n0 = 2 * (wid / ((int64_t)cgroups * p.H));
+  const bool has1 = n0 + 1 < p.n_tokens;  // warp-uniform
   const int d = cg * kRG + lane;
-  const int64_t pos = p.tok_off + n;
-  float acc = 0.f;
+  float acc[2] = {0.f, 0.f};
   for (int t = 0; t < p.T; ++t) {
-    const float r = __fsub_rn(ld_x(p, t, n, h, d), acc);
-    float lo = r, hi = r;
+    float r[2], lo[2], hi[2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      r[u] = (u == 0 || has1) ? __fsub_rn(ld_x(p, t, n0 + u, h, d), acc[u]) : 0.f;
+      lo[u] = hi[u] = r[u];
+    }
 #pragma unroll
     for (int o = 16; o >= 1; o >>= 1) {
-      lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
-      hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        lo[u] = fminf(lo[u], __shfl_xor_sync(0xffffffffu, lo[u], o));
+        hi[u] = fmaxf(hi[u], __shfl_xor_sync(0xffffffffu, hi[u], o));
+      }
     }
-    const __half lo_h = __float2half_rn(lo);
-    const __half sc_h = __float2half_rn(__fdiv_rn(__fsub_rn(hi, lo), 15.f));
-    const float lo32 = __half2float(lo_h), sc32 = __half2float(sc_h);
-    if (lane == 0) p.params[(((int64_t)t * p.H + h) * p.pool + pos) * cgroups + cg] = __halves2half2(lo_h, sc_h);
-    const uint32_t q = q4(r, lo32, sc32);
-    const uint32_t q_odd = __shfl_down_sync(0xffffffffu, q, 1);
-    acc = __fadd_rn(acc, dq4(q, lo32, sc32));
-    if (!(lane & 1)) p.codes[(((int64_t)t * p.H + h) * p.pool + pos) * (p.D / 2) + d / 2] = (uint8_t)(q | (q_odd << 4));
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const __half lo_h = __float2half_rn(lo[u]);
+      const __half sc_h = __float2half_rn(__fdiv_rn(__fsub_rn(hi[u], lo[u]), 15.f));
+      const float lo32 = __half2float(lo_h), sc32 = __half2float(sc_h);
+      const int64_t pos = p.tok_off + n0 + u;
+      const uint32_t q = q4(r[u], lo32, sc32);
+      const uint32_t q_odd = __shfl_down_sync(0xffffffffu, q, 1);
+      acc[u] = __fadd_rn(acc[u], dq4(q, lo32, sc32));
+      if (u == 0 || has1) {
+        if (lane == 0) p.params[(((int64_t)t * p.H + h) * p.pool + pos) * cgroups + cg] = __halves2half2(lo_h, sc_h);
+        if (!(lane & 1)) p.codes[(((int64_t)t * p.H + h) * p.pool + pos) * (p.D / 2) + d / 2] = (uint8_t)(q | (q_odd << 4));
+      }
+    }
   }
 }
 
@@ -568,7 +585,7 @@ extern "C" loopvq_status loopvq_residual_encode(const loopvq_residual_desc* desc
   p.T = g.T; p.H = g.H; p.D = g.D;
   p.codes = codes; p.params = (__half2*)params;
   const int64_t warps = kind == LOOPVQ_KEYS ? ((n_tokens + kRG - 1) / kRG) * g.H * (g.D / 32)
-                                            : n_tokens * g.H * (g.D / kRG);
+                                            : ((n_tokens + 1) / 2) * g.H * (g.D / kRG);
   const int64_t blocks = (warps + 7) / 8;
   if (blocks > 0x7fffffffLL) return LOOPVQ_ERR_UNSUPPORTED;
   cudaStream_t s = (cudaStream_t)stream;
