@@ -94,7 +94,6 @@ __device__ __forceinline__ void umma_commit(uint32_t mbar) {
 }
 __device__ __forceinline__ void tmem_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tmem_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 // Waits for the outstanding TMEM loads and ties r to the wait, so that no use
 // of the loaded registers can be scheduled before it.
 __device__ __forceinline__ void tmem_wait_ld_tied(uint32_t (&r)[32]) {
